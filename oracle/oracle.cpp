@@ -1,0 +1,358 @@
+// Oracle for the fused attention path: a plain, slow, fp64 CPU implementation.
+//
+// TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, includes or calls this
+// file; only the test suite, the smoke check and the benchmark's CPU-baseline leg load it.
+// It shares no code, header or constant with the CUDA path.
+//
+// What it computes, with the passage each part follows:
+//
+//  * Attention(Q,K,V) = softmax(Q K^T * scale) V  -- "FlashAttention on Ascend NPUs",
+//    section on why attention is memory hungry (the formula softmax(QK^T/sqrt(d_k))V).
+//    `oracle_attn_*_rows` evaluate exactly that definition one output row at a time:
+//    scores of the allowed keys, their maximum, the exp-sum, the weighted sum of V rows.
+//  * The naive multi-pass form that stores the whole S x S score matrix -- "Flash
+//    Attention on Ascend: three techniques", section on the memory traffic of standard
+//    attention (scores = QK^T, scale, softmax, probs @ V, each pass through memory).
+//    `oracle_attn_brute` materialises every score matrix and the probability matrix.
+//  * Tiled evaluation with an online softmax -- same page, sections "tiling" (Q blocks in the
+//    outer loop, K/V blocks in the inner loop) and "online softmax" (keep only the running
+//    maximum and running exp-sum; correct earlier partial results when the maximum grows);
+//    "FlashAttention on Ascend NPUs", tiling section (local max and sum, corrected at the
+//    end).  `oracle_attn_tiled` follows those steps with a settable block size.
+//  * MHA/GQA/MQA head mapping -- "FlashAttention variants: GQA, MQA, sparse attention",
+//    section on expanding KV: K and V are repeated along the head axis with
+//    repeat_interleave(Hq/Hkv), so query head h reads KV head floor(h / (Hq/Hkv)).
+//  * Causal and sliding-window masks -- same page, sliding-window section: each token sees
+//    the nearest W tokens, itself included (the prose and the N*W connection count); the
+//    causal mask is aligned to the bottom-right corner when Sq != Skv (the pages are
+//    silent; this is the reading this project takes).  A row with no allowed key returns
+//    O = 0 and LSE = -inf.
+//  * INT8 KV cache used without decompressing it first -- "Flash Attention on Ascend: three
+//    techniques", KV compression section.  The decode oracle evaluates attention over the
+//    dequantised values k_code * k_scale (exact in fp64), one query token per sequence.
+//    With num_splits > 1 it evaluates each key chunk separately and merges the partial
+//    results through their log-sum-exp, the same correction step the online softmax uses.
+//
+// Inputs are bf16 bit patterns (widened exactly to fp64), fp64 arrays, or int8 codes with
+// fp32 scales.  Layouts: Q [B, Sq, Hq, D], K/V [B, Skv, Hkv, D], scales [B, Hkv, Skv],
+// O [B, Sq, Hq, D], LSE [B, Hq, Sq] (natural log).  Rows are addressed as (b, h, i) triples.
+#include <omp.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <vector>
+
+namespace {
+
+const double kNegInf = -std::numeric_limits<double>::infinity();
+
+struct Dims {
+  long B, Hq, Hkv, Sq, Skv, D;
+};
+
+double widen_bf16(uint16_t bits) {
+  uint32_t u = static_cast<uint32_t>(bits) << 16;
+  float f;
+  std::memcpy(&f, &u, sizeof f);
+  return static_cast<double>(f);
+}
+
+// Key j is visible to query row i.  Bottom-right aligned causal mask; a window of W keys
+// that includes the query's own position.
+bool allowed(const Dims& d, int causal, int window, long i, long j) {
+  const long ip = i + d.Skv - d.Sq;
+  if (j < 0 || j >= d.Skv) return false;
+  if (causal && j > ip) return false;
+  if (window > 0 && j <= ip - window) return false;
+  return true;
+}
+
+long kv_head(const Dims& d, long h) { return h / (d.Hq / d.Hkv); }
+
+long q_index(const Dims& d, long b, long i, long h) { return ((b * d.Sq + i) * d.Hq + h) * d.D; }
+long kv_index(const Dims& d, long b, long j, long g) { return ((b * d.Skv + j) * d.Hkv + g) * d.D; }
+
+// One output row by the definition.  Q(idx), K(idx), V(idx) return fp64 elements.
+template <class QF, class KF, class VF>
+void attn_row(const Dims& d, double scale, int causal, int window, long b, long h, long i,
+              long j_begin, long j_end, QF Q, KF K, VF V, double* o, double* lse,
+              std::vector<double>& x) {
+  const long g = kv_head(d, h);
+  x.assign(d.Skv, kNegInf);
+  double m = kNegInf;
+  bool any = false;
+  for (long j = j_begin; j < j_end; ++j) {
+    if (!allowed(d, causal, window, i, j)) continue;
+    double dot = 0.0;
+    const long qi = q_index(d, b, i, h), ki = kv_index(d, b, j, g);
+    for (long t = 0; t < d.D; ++t) dot += Q(qi + t) * K(ki + t);
+    x[j] = scale * dot;
+    if (!any || x[j] > m) m = x[j];
+    any = true;
+  }
+  for (long t = 0; t < d.D; ++t) o[t] = 0.0;
+  if (!any) {
+    *lse = kNegInf;
+    return;
+  }
+  double l = 0.0;
+  for (long j = j_begin; j < j_end; ++j) {
+    if (x[j] == kNegInf) continue;
+    const double p = std::exp(x[j] - m);
+    l += p;
+    const long vi = kv_index(d, b, j, g);
+    for (long t = 0; t < d.D; ++t) o[t] += p * V(vi + t);
+  }
+  for (long t = 0; t < d.D; ++t) o[t] /= l;
+  *lse = m + std::log(l);
+}
+
+bool dims_ok(const Dims& d) {
+  return d.B > 0 && d.Hq > 0 && d.Hkv > 0 && d.Sq > 0 && d.Skv > 0 && d.D > 0 &&
+         d.Hq % d.Hkv == 0;
+}
+
+template <class QF, class KF, class VF>
+int rows_driver(const Dims& d, double scale, int causal, int window, const int64_t* rows,
+                int64_t nrows, double* o, double* lse, int nthreads, QF Q, KF K, VF V) {
+  if (!dims_ok(d) || nrows < 0 || (nrows > 0 && (!rows || !o || !lse))) return -1;
+  for (int64_t r = 0; r < nrows; ++r) {
+    const int64_t b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+    if (b < 0 || b >= d.B || h < 0 || h >= d.Hq || i < 0 || i >= d.Sq) return -1;
+  }
+  if (nthreads <= 0) nthreads = omp_get_max_threads();
+#pragma omp parallel num_threads(nthreads)
+  {
+    std::vector<double> x;
+#pragma omp for schedule(dynamic, 4)
+    for (int64_t r = 0; r < nrows; ++r) {
+      attn_row(d, scale, causal, window, rows[3 * r], rows[3 * r + 1], rows[3 * r + 2], 0, d.Skv,
+               Q, K, V, o + r * d.D, lse + r, x);
+    }
+  }
+  return 0;
+}
+
+}  // namespace
+
+extern "C" {
+
+int oracle_max_threads() { return omp_get_max_threads(); }
+
+// The definition, row by row, on bf16 inputs (bit patterns).  rows: nrows (b, h, i) triples;
+// o: nrows x D; lse: nrows.  Returns 0, or -1 on a bad argument.
+int oracle_attn_bf16_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
+                          int Hkv, int Sq, int Skv, int D, double scale, int causal, int window,
+                          const int64_t* rows, int64_t nrows, double* o, double* lse,
+                          int nthreads) {
+  const Dims d{B, Hq, Hkv, Sq, Skv, D};
+  auto Q = [q](long idx) { return widen_bf16(q[idx]); };
+  auto K = [k](long idx) { return widen_bf16(k[idx]); };
+  auto V = [v](long idx) { return widen_bf16(v[idx]); };
+  return rows_driver(d, scale, causal, window, rows, nrows, o, lse, nthreads, Q, K, V);
+}
+
+// The same definition on fp64 inputs.
+int oracle_attn_f64_rows(const double* q, const double* k, const double* v, int B, int Hq, int Hkv,
+                         int Sq, int Skv, int D, double scale, int causal, int window,
+                         const int64_t* rows, int64_t nrows, double* o, double* lse,
+                         int nthreads) {
+  const Dims d{B, Hq, Hkv, Sq, Skv, D};
+  auto Q = [q](long idx) { return q[idx]; };
+  auto K = [k](long idx) { return k[idx]; };
+  auto V = [v](long idx) { return v[idx]; };
+  return rows_driver(d, scale, causal, window, rows, nrows, o, lse, nthreads, Q, K, V);
+}
+
+// The naive multi-pass form: for every (b, h) build the full Sq x Skv score matrix, scale it,
+// mask it with -inf, softmax each row, multiply by V.  fp64 inputs; all outputs in full layout
+// (O [B,Sq,Hq,D], LSE [B,Hq,Sq]); probs [B,Hq,Sq,Skv] may be null.  Meant for small shapes.
+int oracle_attn_brute(const double* q, const double* k, const double* v, int B, int Hq, int Hkv,
+                      int Sq, int Skv, int D, double scale, int causal, int window, double* o,
+                      double* lse, double* probs) {
+  const Dims d{B, Hq, Hkv, Sq, Skv, D};
+  if (!dims_ok(d) || !q || !k || !v || !o || !lse) return -1;
+  std::vector<double> S(static_cast<size_t>(Sq) * Skv);
+  for (long b = 0; b < B; ++b) {
+    for (long h = 0; h < Hq; ++h) {
+      const long g = kv_head(d, h);
+      // pass 1: scores = Q K^T
+      for (long i = 0; i < Sq; ++i)
+        for (long j = 0; j < Skv; ++j) {
+          double dot = 0.0;
+          for (long t = 0; t < D; ++t) dot += q[q_index(d, b, i, h) + t] * k[kv_index(d, b, j, g) + t];
+          S[i * Skv + j] = dot;
+        }
+      // pass 2: scale, then mask (-inf where a key is not visible)
+      for (long i = 0; i < Sq; ++i)
+        for (long j = 0; j < Skv; ++j) {
+          S[i * Skv + j] *= scale;
+          if (!allowed(d, causal, window, i, j)) S[i * Skv + j] = kNegInf;
+        }
+      // pass 3: row softmax (and the log of its normaliser)
+      for (long i = 0; i < Sq; ++i) {
+        double m = kNegInf;
+        for (long j = 0; j < Skv; ++j) m = std::max(m, S[i * Skv + j]);
+        double* lrow = lse + (b * Hq + h) * Sq + i;
+        if (m == kNegInf) {
+          for (long j = 0; j < Skv; ++j) S[i * Skv + j] = 0.0;
+          *lrow = kNegInf;
+          continue;
+        }
+        double l = 0.0;
+        for (long j = 0; j < Skv; ++j) {
+          S[i * Skv + j] = (S[i * Skv + j] == kNegInf) ? 0.0 : std::exp(S[i * Skv + j] - m);
+          l += S[i * Skv + j];
+        }
+        for (long j = 0; j < Skv; ++j) S[i * Skv + j] /= l;
+        *lrow = m + std::log(l);
+      }
+      if (probs)
+        std::memcpy(probs + (b * Hq + h) * Sq * Skv, S.data(), sizeof(double) * Sq * Skv);
+      // pass 4: output = P V
+      for (long i = 0; i < Sq; ++i)
+        for (long t = 0; t < D; ++t) {
+          double acc = 0.0;
+          for (long j = 0; j < Skv; ++j) acc += S[i * Skv + j] * v[kv_index(d, b, j, g) + t];
+          o[q_index(d, b, i, h) + t] = acc;
+        }
+    }
+  }
+  return 0;
+}
+
+// Tiled evaluation: Q blocks of `tile` rows in the outer loop, K/V blocks of `tile` keys in
+// the inner loop.  Per row only the running maximum m, the running exp-sum l and the
+// unnormalised output are kept; when a block raises the maximum, l and the output are
+// multiplied by exp(m_old - m_new).  fp64 inputs; full-layout outputs.
+int oracle_attn_tiled(const double* q, const double* k, const double* v, int B, int Hq, int Hkv,
+                      int Sq, int Skv, int D, double scale, int causal, int window, int tile,
+                      double* o, double* lse) {
+  const Dims d{B, Hq, Hkv, Sq, Skv, D};
+  if (!dims_ok(d) || tile <= 0 || !q || !k || !v || !o || !lse) return -1;
+  std::vector<double> m(tile), l(tile), acc(static_cast<size_t>(tile) * D), x(tile);
+  for (long b = 0; b < B; ++b) {
+    for (long h = 0; h < Hq; ++h) {
+      const long g = kv_head(d, h);
+      for (long i0 = 0; i0 < Sq; i0 += tile) {
+        const long ni = std::min<long>(tile, Sq - i0);
+        for (long r = 0; r < ni; ++r) {
+          m[r] = kNegInf;
+          l[r] = 0.0;
+          for (long t = 0; t < D; ++t) acc[r * D + t] = 0.0;
+        }
+        for (long j0 = 0; j0 < Skv; j0 += tile) {
+          const long nj = std::min<long>(tile, Skv - j0);
+          for (long r = 0; r < ni; ++r) {
+            const long i = i0 + r;
+            double m_blk = kNegInf;
+            for (long c = 0; c < nj; ++c) {
+              const long j = j0 + c;
+              if (!allowed(d, causal, window, i, j)) {
+                x[c] = kNegInf;
+                continue;
+              }
+              double dot = 0.0;
+              for (long t = 0; t < D; ++t) dot += q[q_index(d, b, i, h) + t] * k[kv_index(d, b, j, g) + t];
+              x[c] = scale * dot;
+              m_blk = std::max(m_blk, x[c]);
+            }
+            if (m_blk == kNegInf) continue;  // nothing visible in this block
+            const double m_new = std::max(m[r], m_blk);
+            const double corr = (m[r] == kNegInf) ? 0.0 : std::exp(m[r] - m_new);
+            l[r] *= corr;
+            for (long t = 0; t < D; ++t) acc[r * D + t] *= corr;
+            for (long c = 0; c < nj; ++c) {
+              if (x[c] == kNegInf) continue;
+              const double p = std::exp(x[c] - m_new);
+              l[r] += p;
+              const long vi = kv_index(d, b, j0 + c, g);
+              for (long t = 0; t < D; ++t) acc[r * D + t] += p * v[vi + t];
+            }
+            m[r] = m_new;
+          }
+        }
+        for (long r = 0; r < ni; ++r) {
+          const long i = i0 + r;
+          double* orow = o + q_index(d, b, i, h);
+          double* lrow = lse + (b * Hq + h) * Sq + i;
+          if (m[r] == kNegInf) {
+            for (long t = 0; t < D; ++t) orow[t] = 0.0;
+            *lrow = kNegInf;
+            continue;
+          }
+          for (long t = 0; t < D; ++t) orow[t] = acc[r * D + t] / l[r];
+          *lrow = m[r] + std::log(l[r]);
+        }
+      }
+    }
+  }
+  return 0;
+}
+
+// Decode over an INT8 KV cache: one query token per sequence (Sq = 1), keys and values
+// dequantised as code * scale.  rows: nrows (b, h) pairs; o: nrows x D; lse: nrows.
+// num_splits = 1 evaluates the definition directly.  num_splits > 1 cuts the keys into
+// chunks of ceil(Skv / num_splits), evaluates each chunk by the definition (giving a
+// normalised partial output O_s and its log-sum-exp L_s) and merges them:
+// L = log sum_s exp(L_s), O = sum_s exp(L_s - L) O_s.
+int oracle_decode_int8_rows(const uint16_t* q, const int8_t* k, const int8_t* v,
+                            const float* k_scale, const float* v_scale, int B, int Hq, int Hkv,
+                            int Skv, int D, double scale, int num_splits, const int64_t* rows,
+                            int64_t nrows, double* o, double* lse, int nthreads) {
+  const Dims d{B, Hq, Hkv, 1, Skv, D};
+  if (!dims_ok(d) || num_splits < 1 || nrows < 0 || (nrows > 0 && (!rows || !o || !lse)))
+    return -1;
+  if (!q || !k || !v || !k_scale || !v_scale) return -1;
+  for (int64_t r = 0; r < nrows; ++r) {
+    if (rows[2 * r] < 0 || rows[2 * r] >= B || rows[2 * r + 1] < 0 || rows[2 * r + 1] >= Hq)
+      return -1;
+  }
+  // Scale of element idx of K/V [B, Skv, Hkv, D] lives at [b, g, j] of [B, Hkv, Skv].
+  auto scale_at = [&d](const float* s, long idx) {
+    const long row = idx / d.D;  // (b * Skv + j) * Hkv + g
+    const long g = row % d.Hkv, bj = row / d.Hkv;
+    const long j = bj % d.Skv, b = bj / d.Skv;
+    return static_cast<double>(s[(b * d.Hkv + g) * d.Skv + j]);
+  };
+  auto Q = [q](long idx) { return widen_bf16(q[idx]); };
+  auto K = [&](long idx) { return static_cast<double>(k[idx]) * scale_at(k_scale, idx); };
+  auto V = [&](long idx) { return static_cast<double>(v[idx]) * scale_at(v_scale, idx); };
+  const long chunk = (Skv + num_splits - 1) / num_splits;
+  if (nthreads <= 0) nthreads = omp_get_max_threads();
+#pragma omp parallel num_threads(nthreads)
+  {
+    std::vector<double> x, part_o(static_cast<size_t>(num_splits) * D), part_l(num_splits);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+      const long b = rows[2 * r], h = rows[2 * r + 1];
+      for (int s = 0; s < num_splits; ++s) {
+        const long j0 = std::min<long>(Skv, s * chunk), j1 = std::min<long>(Skv, (s + 1) * chunk);
+        attn_row(d, scale, 1, 0, b, h, 0, j0, j1, Q, K, V, part_o.data() + s * D, &part_l[s], x);
+      }
+      double mx = kNegInf;
+      for (int s = 0; s < num_splits; ++s) mx = std::max(mx, part_l[s]);
+      double* orow = o + r * D;
+      for (long t = 0; t < D; ++t) orow[t] = 0.0;
+      if (mx == kNegInf) {
+        lse[r] = kNegInf;
+        continue;
+      }
+      double sum = 0.0;
+      for (int s = 0; s < num_splits; ++s)
+        if (part_l[s] != kNegInf) sum += std::exp(part_l[s] - mx);
+      const double L = mx + std::log(sum);
+      for (int s = 0; s < num_splits; ++s) {
+        if (part_l[s] == kNegInf) continue;
+        const double w = std::exp(part_l[s] - L);
+        for (long t = 0; t < D; ++t) orow[t] += w * part_o[s * D + t];
+      }
+      lse[r] = L;
+    }
+  }
+  return 0;
+}
+
+}  // extern "C"

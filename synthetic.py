@@ -1,0 +1,176 @@
+"""Seeded synthetic inputs shared by the tests, the benchmark and the oracle driver.
+
+This module holds no attention arithmetic. It only draws numbers and names workloads:
+
+* ``normal_bf16(seed, n)`` -- a counter-based stream: element pair ``m`` takes the
+  splitmix64 outputs ``2m`` and ``2m+1`` of the generator started at ``seed``, turns
+  them into two uniforms and then into two N(0,1) values by the Box-Muller transform
+  (fp64).  Each value is rounded to fp32 (round-to-nearest-even) and then to bf16
+  (round-to-nearest-even).  The result is returned as raw bf16 bit patterns (uint16).
+* ``quantize_int8_per_token`` -- the INT8 KV-cache recipe of the decode workload:
+  symmetric, one fp32 scale per (token, kv-head) equal to max|x| / 127, codes
+  ``clamp(rint(x / scale), -127, 127)`` with the division in fp32 and ties to even.
+  The pages ("Flash Attention on Ascend: three techniques", section on INT8/INT4 KV
+  compression) state only that the cache is INT8 with the computation done on the
+  compressed data; the per-token symmetric scheme is this project's reading.
+* ``WORKLOADS`` -- the shapes of the pages' examples ("FlashAttention variants: GQA,
+  MQA, sparse attention", benchmark section: seq 4096, 32 query heads, head dim 128;
+  Llama-2-7B 32/32, Mistral-7B 32/8, Falcon-180B 232/1) plus a tiny parity case and
+  an INT8-KV decode case.
+
+Seeds are ``20260 + 10 * workload_index + tensor_index`` with Q=0, K=1, V=2.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+
+import numpy as np
+
+_GAMMA = np.uint64(0x9E3779B97F4A7C15)
+_M1 = np.uint64(0xBF58476D1CE4E5B9)
+_M2 = np.uint64(0x94D049BB133111EB)
+
+
+def splitmix64(seed: int, start: int, count: int) -> np.ndarray:
+    """Outputs ``start .. start+count-1`` of splitmix64 started at state ``seed``."""
+    idx = np.arange(start + 1, start + count + 1, dtype=np.uint64)
+    with np.errstate(over="ignore"):
+        z = np.uint64(seed & 0xFFFFFFFFFFFFFFFF) + idx * _GAMMA
+        z = (z ^ (z >> np.uint64(30))) * _M1
+        z = (z ^ (z >> np.uint64(27))) * _M2
+        z = z ^ (z >> np.uint64(31))
+    return z
+
+
+def normal_f64(seed: int, n: int, chunk: int = 1 << 22) -> np.ndarray:
+    """``n`` N(0,1) draws in fp64 (Box-Muller over splitmix64 pairs)."""
+    out = np.empty(n, dtype=np.float64)
+    npairs = (n + 1) // 2
+    for p0 in range(0, npairs, chunk):
+        p1 = min(npairs, p0 + chunk)
+        raw = splitmix64(seed, 2 * p0, 2 * (p1 - p0)).reshape(-1, 2)
+        a = (raw[:, 0] >> np.uint64(11)).astype(np.float64)
+        b = (raw[:, 1] >> np.uint64(11)).astype(np.float64)
+        u1 = (a + 1.0) * (2.0 ** -53)  # (0, 1]
+        u2 = b * (2.0 ** -53)  # [0, 1)
+        r = np.sqrt(-2.0 * np.log(u1))
+        t = 2.0 * math.pi * u2
+        pair = np.stack([r * np.cos(t), r * np.sin(t)], axis=1).reshape(-1)
+        lo = 2 * p0
+        hi = min(n, 2 * p1)
+        out[lo:hi] = pair[: hi - lo]
+    return out
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """Round fp32 values to bf16 (nearest, ties to even); return uint16 bit patterns."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    rounding = ((u >> np.uint32(16)) & np.uint32(1)) + np.uint32(0x7FFF)
+    with np.errstate(over="ignore"):
+        return ((u + rounding) >> np.uint32(16)).astype(np.uint16)
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def normal_bf16(seed: int, shape) -> np.ndarray:
+    n = int(np.prod(shape))
+    return f32_to_bf16_bits(normal_f64(seed, n).astype(np.float32)).reshape(shape)
+
+
+def quantize_int8_per_token(x_bits: np.ndarray):
+    """bf16 bits ``[B, S, H, D]`` -> (int8 codes ``[B, S, H, D]``, fp32 scales ``[B, H, S]``)."""
+    x = bf16_bits_to_f32(x_bits)
+    amax = np.max(np.abs(x), axis=-1)  # [B, S, H], fp32
+    sc = (amax / np.float32(127.0)).astype(np.float32)
+    safe = np.where(sc > 0, sc, np.float32(1.0)).astype(np.float32)
+    qf = np.rint((x / safe[..., None]).astype(np.float32))
+    q = np.clip(qf, -127, 127).astype(np.int8)
+    q[sc == 0] = 0
+    return q, np.ascontiguousarray(np.transpose(sc, (0, 2, 1)))
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    index: int
+    B: int
+    Hq: int
+    Hkv: int
+    Sq: int
+    Skv: int
+    D: int
+    causal: int
+    window: int = 0
+    int8_kv: bool = False
+    num_splits: int = 1
+    note: str = ""
+
+    @property
+    def scale(self) -> float:
+        """1/sqrt(D) rounded to fp32, the value both sides receive."""
+        return float(np.float32(1.0 / math.sqrt(self.D)))
+
+    def seed(self, tensor_index: int) -> int:
+        return 20260 + 10 * self.index + tensor_index
+
+    def q_shape(self):
+        return (self.B, self.Sq, self.Hq, self.D)
+
+    def kv_shape(self):
+        return (self.B, self.Skv, self.Hkv, self.D)
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", 1, 1, 2, 2, 128, 128, 64, 0,
+                     note="tiny MHA, non-causal, parity only"),
+    "mha_causal": Workload("mha_causal", 2, 2, 32, 32, 4096, 4096, 128, 1,
+                           note="MHA prefill, Llama-2-7B-like heads"),
+    "gqa_causal": Workload("gqa_causal", 3, 1, 32, 8, 4096, 4096, 128, 1,
+                           note="GQA prefill, Mistral-7B-like heads"),
+    "gqa_sw512": Workload("gqa_sw512", 3, 1, 32, 8, 4096, 4096, 128, 1, window=512,
+                          note="GQA prefill with a 512-key sliding window"),
+    "mqa_causal": Workload("mqa_causal", 4, 1, 232, 1, 2048, 2048, 64, 1,
+                           note="MQA prefill, Falcon-180B-like head layout"),
+    "decode_int8": Workload("decode_int8", 5, 16, 32, 8, 1, 32768, 128, 1, int8_kv=True,
+                            num_splits=16, note="GQA decode over an INT8 KV cache"),
+}
+
+
+def make_qkv(w: Workload, q_seed=None, k_seed=None, v_seed=None):
+    """bf16 bit patterns for Q, K, V of a workload (K, V in bf16 before any quantisation)."""
+    q = normal_bf16(w.seed(0) if q_seed is None else q_seed, w.q_shape())
+    k = normal_bf16(w.seed(1) if k_seed is None else k_seed, w.kv_shape())
+    v = normal_bf16(w.seed(2) if v_seed is None else v_seed, w.kv_shape())
+    return q, k, v
+
+
+def make_decode_inputs(w: Workload):
+    """Q bf16 bits [B,1,Hq,D]; K, V int8 [B,Skv,Hkv,D]; k/v scales fp32 [B,Hkv,Skv]."""
+    q, k, v = make_qkv(w)
+    kq, ks = quantize_int8_per_token(k)
+    vq, vs = quantize_int8_per_token(v)
+    return q, kq, vq, ks, vs
+
+
+def sample_rows(B: int, H: int, S: int, seed: int, n_random: int, window: int = 0):
+    """Deterministic row sample (b, h, i): the first and last 64 rows of every (b, h)
+    capped by S, the window edges, and ``n_random`` rows drawn from splitmix64."""
+    fixed = set()
+    edge = [i for i in range(min(64, S))] + [i for i in range(max(0, S - 64), S)]
+    if window > 0:
+        edge += [i for i in (window - 2, window - 1, window, window + 1) if 0 <= i < S]
+    for b in range(B):
+        for h in range(H):
+            for i in edge[:: max(1, len(edge) // 8)]:
+                fixed.add((b, h, i))
+    for b in range(B):
+        fixed.add((b, 0, 0))
+        fixed.add((b, H - 1, S - 1))
+    raw = splitmix64(seed, 0, 3 * n_random).reshape(-1, 3)
+    for r in raw:
+        fixed.add((int(r[0] % np.uint64(B)), int(r[1] % np.uint64(H)), int(r[2] % np.uint64(S))))
+    rows = np.array(sorted(fixed), dtype=np.int64)
+    return rows
