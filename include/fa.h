@@ -1,0 +1,133 @@
+/*
+ * fa.h -- C ABI of the fused tiled attention library (libfa.so, sm_100a).
+ *
+ * The library computes exact scaled-dot-product attention
+ *
+ *     O = softmax(Q K^T * scale + mask) V
+ *
+ * in one fused, tiled pass with an online softmax (running row maximum and row sum, with the
+ * partial output rescaled whenever the maximum grows), so the score matrix never reaches
+ * device memory.  Sources for each piece of the operation:
+ *   - the formula softmax(QK^T / sqrt(d_k)) V and the [batch, seq_len, num_heads, head_dim]
+ *     layout: "FlashAttention on Ascend NPUs", sections on the attention formula and on
+ *     calling the operator (output has the shape of Q);
+ *   - tiling of Q/K/V into blocks and the online softmax that keeps only the current maximum
+ *     and exp-sum per row: "Flash Attention on Ascend: three techniques", sections 1 and 2;
+ *   - MHA/GQA/MQA: query head h reads KV head floor(h / (Hq/Hkv)), the mapping of an explicit
+ *     repeat_interleave of K and V along the head axis, which this library never builds:
+ *     "FlashAttention variants: GQA, MQA, sparse attention", section on expanding KV;
+ *   - causal and sliding-window masks (each query sees its W nearest keys, itself included):
+ *     same page, sliding-window section;
+ *   - decode over an INT8 KV cache computed without decompressing it first: "Flash
+ *     Attention on Ascend: three techniques", section 3 (KV compression).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor arguments are DEVICE pointers owned by the caller, contiguous, 16-byte
+ *     aligned.  The library allocates no device memory in these calls and keeps only host-side
+ *     state (resolved driver entry points and per-device kernel attributes).
+ *   - bf16 tensors are raw IEEE bfloat16 bit patterns; fp32 tensors are IEEE binary32.
+ *   - Calls validate their arguments synchronously and enqueue their kernels asynchronously on
+ *     `stream` (a cudaStream_t; NULL is the legacy default stream).  Errors that happen on the
+ *     device surface at the caller's next synchronisation; fa_device_status() reports the
+ *     library's own device-side failures (a bounded wait that gave up).
+ *   - Thread safety: calls may be made from several host threads; they share no mutable
+ *     state beyond one-time initialisation, which is guarded.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FA_API __attribute__((visibility("default")))
+#else
+#define FA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = -1, /* null pointer, non-positive size, Hq % Hkv != 0, bad window, ... */
+  FA_ERR_UNSUPPORTED = -2, /* head dimension other than 64 or 128 */
+  FA_ERR_ALIGNMENT = -3,   /* a tensor pointer is not 16-byte aligned */
+  FA_ERR_WORKSPACE = -4,   /* decode workspace missing or smaller than required */
+  FA_ERR_CUDA = -5,        /* a CUDA runtime/driver call or a kernel launch failed */
+  FA_ERR_TIMEOUT = -6      /* a kernel gave up a bounded wait (reported by fa_device_status) */
+} fa_status;
+
+/*
+ * Prefill / full forward pass.
+ *   q    bf16 [B, Sq,  Hq,  D]
+ *   k, v bf16 [B, Skv, Hkv, D]
+ *   o    bf16 [B, Sq,  Hq,  D]   written; may not alias q, k or v
+ *   lse  fp32 [B, Hq, Sq]        natural-log log-sum-exp of each row's scaled, masked scores,
+ *                                or NULL to skip it.  A row that sees no key gets O = 0 and
+ *                                LSE = -inf.
+ *   scale   > 0 and finite (1/sqrt(D) for the usual attention).
+ *   causal  0 or 1.  The causal mask is aligned to the bottom-right corner: query i sees key j
+ *           iff j <= i + (Skv - Sq).
+ *   window  <= 0: none.  > 0 (only with causal = 1): query i also needs j > i + (Skv - Sq) -
+ *           window, i.e. it sees its `window` nearest keys including its own position.
+ *   D must be 64 or 128; Hq must be a multiple of Hkv.
+ * Returns FA_OK or an fa_status error code; nothing is launched on error.
+ */
+FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+           int Hkv, int Sq, int Skv, int D, float scale, int causal, int window, void* stream);
+
+/*
+ * Bytes of device workspace fa_decode_int8 needs: fp32 partial outputs [num_splits, B, Hq, D]
+ * followed by fp32 partial log-sum-exps [num_splits, B, Hq], padded to 256 bytes.
+ * Returns 0 for invalid sizes.
+ */
+FA_API size_t fa_decode_int8_workspace_bytes(int B, int Hq, int D, int num_splits);
+
+/*
+ * Decode step (one query token per sequence) over an INT8 KV cache, split over the keys.
+ *   q       bf16 [B, 1, Hq, D]
+ *   k, v    int8 [B, Skv, Hkv, D]   codes; element value = code * scale of its (token, head)
+ *   k_scale, v_scale fp32 [B, Hkv, Skv]
+ *   o       bf16 [B, 1, Hq, D]     written
+ *   lse     fp32 [B, Hq] natural log, or NULL
+ *   num_splits >= 1: the keys are cut into chunks of ceil(Skv / num_splits); each chunk is
+ *           reduced to a partial (output, log-sum-exp) in `workspace`, and a second kernel
+ *           merges the partials through their log-sum-exp.
+ *   workspace  device buffer of at least fa_decode_int8_workspace_bytes(B, Hq, D, num_splits)
+ *           bytes, owned by the caller; its contents on entry do not matter.  Two calls that may
+ *           run concurrently must not share one workspace.
+ * The query sees every key (causal alignment of a single query at the end of the sequence).
+ * D must be 64 or 128; Hq must be a multiple of Hkv.
+ */
+FA_API int fa_decode_int8(const void* q, const int8_t* k, const int8_t* v, const float* k_scale,
+                   const float* v_scale, void* o, float* lse, int B, int Hq, int Hkv, int Skv,
+                   int D, float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                   void* stream);
+
+/* Static, human-readable name of a status code.  Never NULL. */
+FA_API const char* fa_status_string(int status);
+
+/*
+ * Synchronises `stream`, then reads and clears the library's device status word on the current
+ * device.  Returns FA_ERR_TIMEOUT if a kernel launched by this library gave up a bounded wait
+ * since the last call (its outputs are then undefined), FA_ERR_CUDA if the synchronisation
+ * failed, else FA_OK.
+ */
+FA_API int fa_device_status(void* stream);
+
+/*
+ * Diagnostic: launches one thread that waits on a shared-memory barrier nothing ever signals,
+ * with a wall-clock limit of `timeout_us` microseconds (1 .. 10^7).  The wait gives up, records
+ * the timeout in the device status word and the kernel returns normally, so a following
+ * fa_device_status() returns FA_ERR_TIMEOUT.  This exercises the same bounded-wait code every
+ * kernel of the library uses, without faulting or hanging the device.
+ */
+FA_API int fa_selftest_bounded_wait(int timeout_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

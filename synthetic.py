@@ -155,6 +155,79 @@ def make_decode_inputs(w: Workload):
     return q, kq, vq, ks, vs
 
 
+# ---------------------------------------------------------------------------------------
+# The same generator in torch (any device): used for workloads too large to draw in numpy.
+# Integer steps are identical; the fp64 log/cos/sin of the device library may differ from
+# numpy's in the last bit, so a value can (rarely) round to a neighbouring bf16.  Each test or
+# benchmark draws its inputs once and hands the same tensors to both sides.
+# ---------------------------------------------------------------------------------------
+def _i64(u: int) -> int:
+    u &= 0xFFFFFFFFFFFFFFFF
+    return u - (1 << 64) if u >= 1 << 63 else u
+
+
+def _lsr(z, k):
+    import torch
+    return (z >> k) & ((1 << (64 - k)) - 1)
+
+
+def splitmix64_torch(seed: int, start: int, count: int, device="cpu"):
+    import torch
+    idx = torch.arange(start + 1, start + count + 1, dtype=torch.int64, device=device)
+    z = idx * _i64(0x9E3779B97F4A7C15) + _i64(seed)
+    z = (z ^ _lsr(z, 30)) * _i64(0xBF58476D1CE4E5B9)
+    z = (z ^ _lsr(z, 27)) * _i64(0x94D049BB133111EB)
+    return z ^ _lsr(z, 31)
+
+
+def normal_bf16_torch(seed: int, shape, device="cpu", chunk: int = 1 << 24):
+    """bf16 tensor of N(0,1) draws from the same stream as ``normal_bf16``."""
+    import torch
+    n = int(np.prod(shape))
+    out = torch.empty(n, dtype=torch.bfloat16, device=device)
+    npairs = (n + 1) // 2
+    for p0 in range(0, npairs, chunk):
+        p1 = min(npairs, p0 + chunk)
+        raw = splitmix64_torch(seed, 2 * p0, 2 * (p1 - p0), device).view(-1, 2)
+        a = _lsr(raw[:, 0], 11).to(torch.float64)
+        b = _lsr(raw[:, 1], 11).to(torch.float64)
+        u1 = (a + 1.0) * (2.0 ** -53)
+        u2 = b * (2.0 ** -53)
+        r = torch.sqrt(-2.0 * torch.log(u1))
+        t = (2.0 * math.pi) * u2
+        pair = torch.stack([r * torch.cos(t), r * torch.sin(t)], dim=1).reshape(-1)
+        lo, hi = 2 * p0, min(n, 2 * p1)
+        out[lo:hi] = pair[: hi - lo].to(torch.float32).to(torch.bfloat16)
+        del raw, a, b, u1, u2, r, t, pair
+    return out.view(*shape)
+
+
+def quantize_int8_per_token_torch(x):
+    """torch version of ``quantize_int8_per_token``: bf16 [B,S,H,D] -> (int8 [B,S,H,D],
+    fp32 scales [B,H,S])."""
+    import torch
+    xf = x.to(torch.float32)
+    amax = xf.abs().amax(dim=-1)
+    sc = amax / 127.0
+    safe = torch.where(sc > 0, sc, torch.ones_like(sc))
+    q = torch.clamp(torch.round(xf / safe[..., None]), -127, 127).to(torch.int8)
+    q[sc == 0] = 0
+    return q, sc.permute(0, 2, 1).contiguous()
+
+
+def make_qkv_torch(w: Workload, device):
+    return (normal_bf16_torch(w.seed(0), w.q_shape(), device),
+            normal_bf16_torch(w.seed(1), w.kv_shape(), device),
+            normal_bf16_torch(w.seed(2), w.kv_shape(), device))
+
+
+def make_decode_inputs_torch(w: Workload, device):
+    q = normal_bf16_torch(w.seed(0), w.q_shape(), device)
+    kq, ks = quantize_int8_per_token_torch(normal_bf16_torch(w.seed(1), w.kv_shape(), device))
+    vq, vs = quantize_int8_per_token_torch(normal_bf16_torch(w.seed(2), w.kv_shape(), device))
+    return q, kq, vq, ks, vs
+
+
 def sample_rows(B: int, H: int, S: int, seed: int, n_random: int, window: int = 0):
     """Deterministic row sample (b, h, i): the first and last 64 rows of every (b, h)
     capped by S, the window edges, and ``n_random`` rows drawn from splitmix64."""

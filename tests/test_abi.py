@@ -1,0 +1,118 @@
+"""Host-only checks of the C ABI: the library loads without a GPU, exports every function that
+include/fa.h declares, and rejects bad arguments with the documented status codes before it
+touches the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import tiled_attention_26_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails before any CUDA call
+
+
+@pytest.fixture(scope="module")
+def L():
+    from tiled_attention_26_b200 import build
+    build.build()
+    return fa.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*FA_API\s+(?:const\s+)?\w+\s*\*?\s*(fa_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("fa_fwd", "fa_decode_int8", "fa_decode_int8_workspace_bytes", "fa_status_string",
+              "fa_device_status", "fa_selftest_bounded_wait"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_codes_match_header():
+    text = open(HEADER).read()
+    for name, value in fa.STATUS.items():
+        assert re.search(rf"\b{name}\s*=\s*{value}\b", text), name
+
+
+def test_status_strings(L):
+    for name, value in fa.STATUS.items():
+        assert fa.fa_status_string(value).startswith(name)
+    assert fa.fa_status_string(12345) == "unknown fa_status"
+
+
+def fwd(L, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, Hq=2, Hkv=2, Sq=128, Skv=128, D=64,
+        scale=0.125, causal=0, window=0):
+    return L.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, window, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(o=None), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(B=0), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(Sq=-1), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(Hq=6, Hkv=4), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(window=16), fa.STATUS["FA_ERR_INVALID_ARG"]),          # window needs causal
+    (dict(window=-1, causal=1), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(causal=2), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(scale=0.0), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(scale=float("nan")), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(scale=float("inf")), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(D=96), fa.STATUS["FA_ERR_UNSUPPORTED"]),
+    (dict(D=256), fa.STATUS["FA_ERR_UNSUPPORTED"]),
+    (dict(q=FAKE + 8), fa.STATUS["FA_ERR_ALIGNMENT"]),
+    (dict(o=FAKE + 2), fa.STATUS["FA_ERR_ALIGNMENT"]),
+    (dict(lse=FAKE + 1), fa.STATUS["FA_ERR_ALIGNMENT"]),
+])
+def test_fwd_rejects(L, kw, code):
+    assert fwd(L, **kw) == code
+
+
+def dec(L, q=FAKE, k=FAKE, v=FAKE, ks=FAKE, vs=FAKE, o=FAKE, lse=None, B=2, Hq=8, Hkv=2, Skv=100,
+        D=128, scale=0.1, splits=4, ws=FAKE, ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = L.fa_decode_int8_workspace_bytes(B, Hq, D, splits)
+    return L.fa_decode_int8(q, k, v, ks, vs, o, lse, B, Hq, Hkv, Skv, D, scale, splits, ws,
+                            ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=None), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(vs=None), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(splits=0), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(Skv=0), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(Hq=6, Hkv=4), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(scale=-1.0), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(D=80), fa.STATUS["FA_ERR_UNSUPPORTED"]),
+    (dict(ks=FAKE + 4), fa.STATUS["FA_ERR_ALIGNMENT"]),
+    (dict(ws=None), fa.STATUS["FA_ERR_WORKSPACE"]),
+    (dict(ws_bytes=16), fa.STATUS["FA_ERR_WORKSPACE"]),
+])
+def test_decode_rejects(L, kw, code):
+    assert dec(L, **kw) == code
+
+
+def test_workspace_bytes(L):
+    B, Hq, D, S = 16, 32, 128, 16
+    o_bytes = S * B * Hq * D * 4
+    lse_bytes = S * B * Hq * 4
+    got = fa.fa_decode_int8_workspace_bytes(B, Hq, D, S)
+    assert got >= o_bytes + lse_bytes and got % 256 == 0 and got - (o_bytes + lse_bytes) < 512
+    assert fa.fa_decode_int8_workspace_bytes(0, Hq, D, S) == 0
+    assert fa.fa_decode_int8_workspace_bytes(B, Hq, D, 0) == 0
+
+
+def test_selftest_rejects_bad_timeout(L):
+    assert L.fa_selftest_bounded_wait(0, None) == fa.STATUS["FA_ERR_INVALID_ARG"]
+    assert L.fa_selftest_bounded_wait(10 ** 8, None) == fa.STATUS["FA_ERR_INVALID_ARG"]

@@ -55,3 +55,17 @@ def test_workload_table():
     d = w["decode_int8"]
     assert (d.B, d.Hq, d.Hkv, d.Sq, d.Skv, d.num_splits) == (16, 32, 8, 1, 32768, 16)
     assert w["tiny"].scale == 0.125
+
+
+def test_torch_generator_matches_numpy_stream():
+    import torch
+    ints = synthetic.splitmix64_torch(1234567, 0, 5)
+    assert [int(x) & 0xFFFFFFFFFFFFFFFF for x in ints] == [int(x) for x in synthetic.splitmix64(1234567, 0, 5)]
+    a = synthetic.normal_bf16(777, (3, 1001))
+    b = synthetic.normal_bf16_torch(777, (3, 1001), chunk=257).view(torch.int16).numpy().view(np.uint16)
+    # same integer stream; fp64 transcendental functions may differ in the last bit
+    assert np.mean(a != b) < 1e-3
+    q1, s1 = synthetic.quantize_int8_per_token(a.reshape(1, 3, 7, 143))
+    tq, ts = synthetic.quantize_int8_per_token_torch(
+        torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).reshape(1, 3, 7, 143))
+    assert np.array_equal(q1, tq.numpy()) and np.array_equal(s1, ts.numpy())

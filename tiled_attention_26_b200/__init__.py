@@ -1,0 +1,173 @@
+"""Python binding of ``libfa.so``, the fused tiled attention library for B200 (sm_100a).
+
+The functions carry the C names of ``include/fa.h`` and only marshal arguments: they check
+dtypes, shapes and devices of torch tensors, allocate outputs when none are given (torch is the
+device-memory allocator here), and pass raw pointers and sizes to the C ABI.  Every step of the
+computation runs in the library's CUDA kernels.  If ``libfa.so`` is missing or cannot be loaded,
+every call raises; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+__all__ = ["FaError", "lib", "fa_fwd", "fa_decode_int8", "fa_decode_int8_workspace_bytes",
+           "fa_status_string", "fa_device_status", "fa_selftest_bounded_wait", "LIB_PATH",
+           "STATUS"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
+
+STATUS = {
+    "FA_OK": 0,
+    "FA_ERR_INVALID_ARG": -1,
+    "FA_ERR_UNSUPPORTED": -2,
+    "FA_ERR_ALIGNMENT": -3,
+    "FA_ERR_WORKSPACE": -4,
+    "FA_ERR_CUDA": -5,
+    "FA_ERR_TIMEOUT": -6,
+}
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {fa_status_string(status)} ({status})")
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_Z = ctypes.c_size_t
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library, with argument types declared.  Raises if it is not built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"libfa.so is not built ({LIB_PATH}); run "
+                               "`python tiled_attention_26_b200/build.py`")
+        L = ctypes.CDLL(LIB_PATH)
+        L.fa_fwd.argtypes = [_P, _P, _P, _P, _P] + [_I] * 6 + [_F, _I, _I, _P]
+        L.fa_fwd.restype = _I
+        L.fa_decode_int8_workspace_bytes.argtypes = [_I, _I, _I, _I]
+        L.fa_decode_int8_workspace_bytes.restype = _Z
+        L.fa_decode_int8.argtypes = [_P] * 7 + [_I] * 5 + [_F, _I, _P, _Z, _P]
+        L.fa_decode_int8.restype = _I
+        L.fa_status_string.argtypes = [_I]
+        L.fa_status_string.restype = ctypes.c_char_p
+        L.fa_device_status.argtypes = [_P]
+        L.fa_device_status.restype = _I
+        L.fa_selftest_bounded_wait.argtypes = [_I, _P]
+        L.fa_selftest_bounded_wait.restype = _I
+        _lib = L
+    return _lib
+
+
+def fa_status_string(status: int) -> str:
+    return lib().fa_status_string(int(status)).decode()
+
+
+def _stream_ptr(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(t, name, dtype, shape, device):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def fa_fwd(q, k, v, causal: bool = False, window: int = 0, scale: float | None = None,
+           o=None, lse=None, return_lse: bool = True, stream=None):
+    """Attention forward.  q: bf16 [B, Sq, Hq, D] on CUDA; k, v: bf16 [B, Skv, Hkv, D].
+
+    Returns ``(o, lse)``: o bf16 [B, Sq, Hq, D], lse fp32 [B, Hq, Sq] (natural log; None when
+    ``return_lse`` is false and no ``lse`` buffer is given)."""
+    import torch
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q, k, v must be 4-D [B, S, H, D]")
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    dev = q.device
+    _check(q, "q", torch.bfloat16, (B, Sq, Hq, D), dev)
+    _check(k, "k", torch.bfloat16, (B, Skv, Hkv, D), dev)
+    _check(v, "v", torch.bfloat16, (B, Skv, Hkv, D), dev)
+    if o is None:
+        o = torch.empty_like(q)
+    _check(o, "o", torch.bfloat16, (B, Sq, Hq, D), dev)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq, Sq), dtype=torch.float32, device=dev)
+    if lse is not None:
+        _check(lse, "lse", torch.float32, (B, Hq, Sq), dev)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                      lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Sq, Skv, D,
+                      float(scale), int(bool(causal)), int(window), _stream_ptr(stream))
+    if rc != 0:
+        raise FaError(rc, "fa_fwd")
+    return o, lse
+
+
+def fa_decode_int8_workspace_bytes(B: int, Hq: int, D: int, num_splits: int) -> int:
+    return int(lib().fa_decode_int8_workspace_bytes(int(B), int(Hq), int(D), int(num_splits)))
+
+
+def fa_decode_int8(q, k, v, k_scale, v_scale, num_splits: int = 16, scale: float | None = None,
+                   o=None, lse=None, workspace=None, return_lse: bool = True, stream=None):
+    """Decode step over an INT8 KV cache.  q: bf16 [B, 1, Hq, D]; k, v: int8 [B, Skv, Hkv, D];
+    k_scale, v_scale: fp32 [B, Hkv, Skv].  Returns ``(o, lse)`` with o bf16 [B, 1, Hq, D] and
+    lse fp32 [B, Hq]."""
+    import torch
+    B, one, Hq, D = q.shape
+    if one != 1:
+        raise ValueError("decode takes one query token per sequence")
+    Skv, Hkv = k.shape[1], k.shape[2]
+    dev = q.device
+    _check(q, "q", torch.bfloat16, (B, 1, Hq, D), dev)
+    _check(k, "k", torch.int8, (B, Skv, Hkv, D), dev)
+    _check(v, "v", torch.int8, (B, Skv, Hkv, D), dev)
+    _check(k_scale, "k_scale", torch.float32, (B, Hkv, Skv), dev)
+    _check(v_scale, "v_scale", torch.float32, (B, Hkv, Skv), dev)
+    if o is None:
+        o = torch.empty_like(q)
+    _check(o, "o", torch.bfloat16, (B, 1, Hq, D), dev)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    if lse is not None:
+        _check(lse, "lse", torch.float32, (B, Hq), dev)
+    need = fa_decode_int8_workspace_bytes(B, Hq, D, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    rc = lib().fa_decode_int8(q.data_ptr(), k.data_ptr(), v.data_ptr(), k_scale.data_ptr(),
+                              v_scale.data_ptr(), o.data_ptr(),
+                              lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Skv, D,
+                              float(scale), int(num_splits), workspace.data_ptr(),
+                              workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    if rc != 0:
+        raise FaError(rc, "fa_decode_int8")
+    return o, lse
+
+
+def fa_device_status(stream=None) -> int:
+    return int(lib().fa_device_status(_stream_ptr(stream)))
+
+
+def fa_selftest_bounded_wait(timeout_us: int, stream=None) -> int:
+    return int(lib().fa_selftest_bounded_wait(int(timeout_us), _stream_ptr(stream)))

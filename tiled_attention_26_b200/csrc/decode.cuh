@@ -1,0 +1,381 @@
+// Split-KV decode over an INT8 KV cache, plus the kernel that merges the splits.
+//
+// One query token per sequence attends to Skv cached keys whose K and V are stored as int8
+// codes with one fp32 scale per (token, KV head).  The codes are used directly ("Flash
+// Attention on Ascend: three techniques", section 3: the compressed cache takes part in the
+// computation without being decompressed first):
+//   score_j = scale * k_scale_j * (q . kcode_j)          O = sum_j p_j * v_scale_j * vcode_j
+// so the scales leave the dot products and each code converts exactly to fp16.
+//
+// Split step (fa_decode_split_kernel): one CTA per (split, batch, KV head, block of <= 8 query
+// heads of that KV head's group); 4 warps stride over the split's keys 32 at a time.  Each warp
+// streams the int8 rows straight from HBM into registers with 16-byte non-caching loads,
+// converts them to fp16 with byte permutes and one fp16 subtract, and runs both contractions on
+// the tensor cores with mma.sync m16n8k16 (fp32 accumulate):
+//   S  = Kcode[16 tokens x 16 dims] . Q^T[16 dims x 8 heads]   (tokens as M, heads as N)
+//   O^T += Vcode^T[16 dims x 16 tokens] . P'^T[16 tokens x 8 heads]
+// The reduction index of each contraction is permuted (dims for QK, dims of the output rows
+// for PV) so that every thread's fragment comes from contiguous bytes of one row; Q and the
+// output use the same permutations, so the results are unchanged.  P' = p * v_scale is moved
+// from the QK accumulator layout into the PV operand layout with movmatrix (8x8 transpose).
+// The online softmax (running max m and sum l per head, rescale when m grows by more than 2^8)
+// runs on the accumulator fragments.  The 4 warps merge through shared memory and the CTA
+// writes a normalised partial output and its log-sum-exp to the workspace.
+//
+// Merge step (fa_decode_combine_kernel): L = log sum_s exp(L_s), O = sum_s exp(L_s - L) O_s.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace fa {
+
+struct DecodeParams {
+  const uint16_t* q;  // bf16 [B, 1, Hq, D]
+  const int8_t* k;    // [B, Skv, Hkv, D]
+  const int8_t* v;
+  const float* k_scale;  // [B, Hkv, Skv]
+  const float* v_scale;
+  float* o_part;    // [splits, B, Hq, D]
+  float* lse_part;  // [splits, B, Hq]
+  int B, Hq, Hkv, Skv, G, splits, chunk;
+  float scale_log2;
+};
+
+struct CombineParams {
+  const float* o_part;
+  const float* lse_part;
+  uint16_t* o;  // bf16 [B, 1, Hq, D]
+  float* lse;   // [B, Hq] or null
+  int B, Hq, splits;
+};
+
+__device__ __forceinline__ uint4 ldg_stream16(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint2 ldg_stream8(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+               : "=r"(r.x), "=r"(r.y)
+               : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+// Two biased bytes (x + 128) in the low bytes of a fp16 pair with exponent 2^10 give
+// 1024 + x + 128 exactly; subtracting 1152 leaves x exactly.
+constexpr uint32_t kMagic64 = 0x64646464u;
+__device__ __forceinline__ uint32_t f16x2_minus_1152(uint32_t h) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(h), "r"(0x64806480u));
+  return d;
+}
+// bytes (x0, x1) at byte positions (lo, lo+1) of a biased word -> fp16x2 {x0, x1}
+__device__ __forceinline__ uint32_t codes_to_f16x2(uint32_t biased, uint32_t sel) {
+  return f16x2_minus_1152(prmt(biased, kMagic64, sel));
+}
+constexpr uint32_t kSelB01 = 0x4140u;  // [b0, 0x64, b1, 0x64]
+constexpr uint32_t kSelB23 = 0x4342u;  // [b2, 0x64, b3, 0x64]
+
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                              uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+// Power of two 2^e with e chosen so that x * 2^e < 2^top (x > 0), clamped to a safe range.
+__device__ __forceinline__ int pow2_exponent_below(float x, int top) {
+  if (!(x > 0.f)) return 0;
+  int ex;
+  frexpf(x, &ex);  // x = f * 2^ex, f in [0.5, 1): x < 2^ex
+  return max(-100, min(100, top - ex));
+}
+
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) << 23); }
+
+template <int D>
+__global__ void __launch_bounds__(128) fa_decode_split_kernel(const DecodeParams p) {
+  constexpr int KS = D / 16;  // QK k-steps
+  constexpr int MT = D / 16;  // PV m-tiles (16 output dims each)
+  constexpr int VB = D / 8;   // V bytes per thread per token
+  const int split = blockIdx.x;
+  const int b = blockIdx.y / p.Hkv, kvh = blockIdx.y % p.Hkv;
+  const int head0 = kvh * p.G + blockIdx.z * 8;
+  const int nheads = min(8, p.G - static_cast<int>(blockIdx.z) * 8);
+  const int t_begin = split * p.chunk;
+  const int t_end = min(p.Skv, t_begin + p.chunk);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+
+  __shared__ float sm_red[4];
+  __shared__ float sm_m[4][8], sm_l[4][8];
+  __shared__ float sm_o[4][8][D];
+
+  const float* ks_row = p.k_scale + (static_cast<size_t>(b) * p.Hkv + kvh) * p.Skv;
+  const float* vs_row = p.v_scale + (static_cast<size_t>(b) * p.Hkv + kvh) * p.Skv;
+
+  // ---- P' = p * v_scale * 2^E stays below 2^15 in fp16: E from the split's largest v_scale ----
+  float vmax = 0.f;
+  for (int t = t_begin + threadIdx.x; t < t_end; t += 128) vmax = fmaxf(vmax, vs_row[t]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+  if (lane == 0) sm_red[warp] = vmax;
+  __syncthreads();
+  vmax = fmaxf(fmaxf(sm_red[0], sm_red[1]), fmaxf(sm_red[2], sm_red[3]));
+  const int E = pow2_exponent_below(vmax, 7);  // p <= 2^8 with the lazy rescale
+  const float pscale = exp2i(E);
+
+  // ---- Q as the B operand of the QK mma, fp16, scaled by 2^eq per head (exact) ----
+  uint32_t qf[KS][2];
+  float sc_mine;
+  {
+    float qv[KS][4];
+    const bool hv = g < nheads;
+    const uint16_t* qrow = p.q + (static_cast<size_t>(b) * p.Hq + head0 + (hv ? g : 0)) * D;
+    float amax = 0.f;
+#pragma unroll
+    for (int s = 0; s < KS; ++s)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int dim = (s / 4) * 64 + 16 * c + 4 * (s % 4) + e;
+        qv[s][e] = hv ? bf16_bits_to_float(qrow[dim]) : 0.f;
+        amax = fmaxf(amax, fabsf(qv[s][e]));
+      }
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    const int eq = pow2_exponent_below(amax, 15);
+    const float qs = exp2i(eq);
+#pragma unroll
+    for (int s = 0; s < KS; ++s) {
+      qf[s][0] = pack_f16x2(qv[s][0] * qs, qv[s][1] * qs);
+      qf[s][1] = pack_f16x2(qv[s][2] * qs, qv[s][3] * qs);
+    }
+    sc_mine = p.scale_log2 * exp2i(-eq);
+  }
+  // this thread's accumulator columns are heads 2c and 2c+1
+  const float sc0 = __shfl_sync(0xffffffffu, sc_mine, 8 * c);
+  const float sc1 = __shfl_sync(0xffffffffu, sc_mine, 8 * c + 4);
+
+  float oacc[MT][4];
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) oacc[mt][0] = oacc[mt][1] = oacc[mt][2] = oacc[mt][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+  const size_t row_stride = static_cast<size_t>(p.Hkv) * D;  // bytes between tokens
+  const int8_t* kbase = p.k + (static_cast<size_t>(b) * p.Skv * p.Hkv + kvh) * D;
+  const int8_t* vbase = p.v + (static_cast<size_t>(b) * p.Skv * p.Hkv + kvh) * D;
+  const int nsteps = (t_end - t_begin + 31) / 32;
+
+  for (int st = warp; st < nsteps; st += 4) {
+    const int T = t_begin + 32 * st;
+    // -- loads (rows past the end are clamped for the address and masked below) --
+    uint32_t kw[2][2][KS];  // [group][row g / g+8][k-step]
+    uint32_t vw[2][4][VB / 4];
+    float ksc[2][2], vsc[2][2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const int tok = min(T + 16 * u + g + 8 * rr, p.Skv - 1);
+        const int8_t* row = kbase + static_cast<size_t>(tok) * row_stride;
+        const uint4 lo = ldg_stream16(row + 16 * c);
+        kw[u][rr][0] = lo.x;
+        kw[u][rr][1] = lo.y;
+        kw[u][rr][2] = lo.z;
+        kw[u][rr][3] = lo.w;
+        if constexpr (D == 128) {
+          const uint4 hi = ldg_stream16(row + 64 + 16 * c);
+          kw[u][rr][4 % KS] = hi.x;
+          kw[u][rr][5 % KS] = hi.y;
+          kw[u][rr][6 % KS] = hi.z;
+          kw[u][rr][7 % KS] = hi.w;
+        }
+        ksc[u][rr] = ks_row[tok];
+        vsc[u][rr] = vs_row[tok];
+      }
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const int tok = min(T + 16 * u + 2 * c + (q4 & 1) + 8 * (q4 >> 1), p.Skv - 1);
+        const int8_t* row = vbase + static_cast<size_t>(tok) * row_stride + VB * g;
+        if constexpr (VB == 16) {
+          const uint4 x = ldg_stream16(row);
+          vw[u][q4][0] = x.x;
+          vw[u][q4][1 % (VB / 4)] = x.y;
+          vw[u][q4][2 % (VB / 4)] = x.z;
+          vw[u][q4][3 % (VB / 4)] = x.w;
+        } else {
+          const uint2 x = ldg_stream8(row);
+          vw[u][q4][0] = x.x;
+          vw[u][q4][1 % (VB / 4)] = x.y;
+        }
+      }
+    }
+
+    // -- S = Kcode . Q^T per 16-token group; x = score in log2 units --
+    float x[2][4];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int s = 0; s < KS; ++s) {
+        const uint32_t w0 = kw[u][0][s] ^ 0x80808080u, w1 = kw[u][1][s] ^ 0x80808080u;
+        mma_f16_16816(sacc, codes_to_f16x2(w0, kSelB01), codes_to_f16x2(w1, kSelB01),
+                      codes_to_f16x2(w0, kSelB23), codes_to_f16x2(w1, kSelB23), qf[s][0],
+                      qf[s][1]);
+      }
+      const int tA = T + 16 * u + g, tB = tA + 8;
+      x[u][0] = tA < t_end ? sacc[0] * ksc[u][0] * sc0 : -INFINITY;
+      x[u][1] = tA < t_end ? sacc[1] * ksc[u][0] * sc1 : -INFINITY;
+      x[u][2] = tB < t_end ? sacc[2] * ksc[u][1] * sc0 : -INFINITY;
+      x[u][3] = tB < t_end ? sacc[3] * ksc[u][1] * sc1 : -INFINITY;
+    }
+
+    // -- online softmax per head (columns 2c, 2c+1); max over the warp's 32 tokens --
+    float mx0 = fmaxf(fmaxf(x[0][0], x[0][2]), fmaxf(x[1][0], x[1][2]));
+    float mx1 = fmaxf(fmaxf(x[0][1], x[0][3]), fmaxf(x[1][1], x[1][3]));
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    if (mx0 > m0 + 8.f) {
+      const float a = ex2(m0 - mx0);
+      m0 = mx0;
+      l0 *= a;
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        oacc[mt][0] *= a;
+        oacc[mt][2] *= a;
+      }
+    }
+    if (mx1 > m1 + 8.f) {
+      const float a = ex2(m1 - mx1);
+      m1 = mx1;
+      l1 *= a;
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        oacc[mt][1] *= a;
+        oacc[mt][3] *= a;
+      }
+    }
+    const float mu0 = (m0 == -INFINITY) ? 0.f : m0;
+    const float mu1 = (m1 == -INFINITY) ? 0.f : m1;
+    uint32_t pb[2][2];  // PV B operand per group: tokens 0-7 and 8-15 of the group
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float pa0 = ex2(x[u][0] - mu0), pa1 = ex2(x[u][1] - mu1);
+      const float pb0 = ex2(x[u][2] - mu0), pb1 = ex2(x[u][3] - mu1);
+      l0 += pa0 + pb0;
+      l1 += pa1 + pb1;
+      const float wa = vsc[u][0] * pscale, wb = vsc[u][1] * pscale;
+      pb[u][0] = movmatrix_trans(pack_f16x2(pa0 * wa, pa1 * wa));
+      pb[u][1] = movmatrix_trans(pack_f16x2(pb0 * wb, pb1 * wb));
+    }
+
+    // -- O^T += Vcode^T . P'^T --
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      uint32_t r[4][VB / 4];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4)
+#pragma unroll
+        for (int w = 0; w < VB / 4; ++w) r[q4][w] = vw[u][q4][w] ^ 0x80808080u;
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        const int w = mt >> 1;
+        const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
+        const uint32_t x01 = prmt(r[0][w], r[1][w], sel);  // tokens 2c, 2c+1
+        const uint32_t x89 = prmt(r[2][w], r[3][w], sel);  // tokens 2c+8, 2c+9
+        mma_f16_16816(oacc[mt], codes_to_f16x2(x01, kSelB01), codes_to_f16x2(x01, kSelB23),
+                      codes_to_f16x2(x89, kSelB01), codes_to_f16x2(x89, kSelB23), pb[u][0],
+                      pb[u][1]);
+      }
+    }
+  }
+
+  // ---- merge the 4 warps ----
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+  }
+  if (g == 0) {
+    sm_m[warp][2 * c] = m0;
+    sm_m[warp][2 * c + 1] = m1;
+    sm_l[warp][2 * c] = l0;
+    sm_l[warp][2 * c + 1] = l1;
+  }
+#pragma unroll
+  for (int mt = 0; mt < MT; ++mt) {
+    const int d0 = VB * g + 2 * mt;
+    sm_o[warp][2 * c][d0] = oacc[mt][0];
+    sm_o[warp][2 * c + 1][d0] = oacc[mt][1];
+    sm_o[warp][2 * c][d0 + 1] = oacc[mt][2];
+    sm_o[warp][2 * c + 1][d0 + 1] = oacc[mt][3];
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < nheads * D; idx += 128) {
+    const int h = idx / D, d = idx % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, sm_m[w][h]);
+    float L = 0.f, acc = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float f = (sm_m[w][h] == -INFINITY) ? 0.f : ex2(sm_m[w][h] - M);
+        L += f * sm_l[w][h];
+        acc += f * sm_o[w][h][d];
+      }
+    }
+    const size_t row = (static_cast<size_t>(split) * p.B + b) * p.Hq + head0 + h;
+    p.o_part[row * D + d] = (L > 0.f) ? acc / (L * pscale) : 0.f;
+    if (d == 0) p.lse_part[row] = (L > 0.f) ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(D) fa_decode_combine_kernel(const CombineParams p) {
+  const int bh = blockIdx.x;
+  const int d = threadIdx.x;
+  float M = -INFINITY;
+  for (int s = 0; s < p.splits; ++s)
+    M = fmaxf(M, p.lse_part[static_cast<size_t>(s) * p.B * p.Hq + bh]);
+  float L = 0.f, acc = 0.f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < p.splits; ++s) {
+      const float ls = p.lse_part[static_cast<size_t>(s) * p.B * p.Hq + bh];
+      if (ls == -INFINITY) continue;
+      const float w = expf(ls - M);
+      L += w;
+      acc += w * p.o_part[(static_cast<size_t>(s) * p.B * p.Hq + bh) * D + d];
+    }
+  }
+  const float o = (L > 0.f) ? acc / L : 0.f;
+  p.o[static_cast<size_t>(bh) * D + d] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+  if (d == 0 && p.lse != nullptr) p.lse[bh] = (L > 0.f) ? M + logf(L) : -INFINITY;
+}
+
+}  // namespace fa

@@ -1,0 +1,254 @@
+// Host side of libfa.so: argument validation, TMA descriptor encoding and kernel launches for
+// the entry points declared in include/fa.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/fa.h"
+#include "decode.cuh"
+#include "prefill.cuh"
+#include "sm100.cuh"
+
+namespace {
+
+constexpr uint64_t kKernelTimeoutNs = 4000000000ull;  // bounded waits give up after 4 s
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// 4-D bf16 tensor [n3][n2][n1][n0] (n0 innermost), boxes of (64, b1, b2, 1), 128-byte swizzle.
+int encode_bf16_4d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1, uint64_t n2,
+                   uint64_t n3, uint32_t b1, uint32_t b2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return FA_ERR_CUDA;
+  const cuuint64_t dims[4] = {n0, n1, n2, n3};
+  const cuuint64_t strides[3] = {n0 * 2, n0 * n1 * 2, n0 * n1 * n2 * 2};
+  const cuuint32_t box[4] = {64, b1, b2, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+template <class Kernel>
+int ensure_smem_attr(Kernel kernel, int bytes, std::atomic<uint64_t>& done_mask) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FA_ERR_CUDA;
+  const uint64_t bit = uint64_t(1) << dev;
+  if (done_mask.load(std::memory_order_acquire) & bit) return FA_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return FA_ERR_CUDA;
+  done_mask.fetch_or(bit, std::memory_order_acq_rel);
+  return FA_OK;
+}
+
+std::atomic<uint64_t> g_attr_prefill64{0}, g_attr_prefill128{0};
+
+template <int D>
+int launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                   int Hkv, int Sq, int Skv, float scale, int causal, int window,
+                   cudaStream_t stream) {
+  using C = fa::PrefillCfg<D>;
+  fa::PrefillParams p{};
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Sq = Sq;
+  p.Skv = Skv;
+  p.G = Hq / Hkv;
+  p.Gp = 1;
+  while (p.Gp < 8 && p.G % (2 * p.Gp) == 0) p.Gp *= 2;
+  p.NP = p.G / p.Gp;
+  const int tokens_per_cta = 256 / p.Gp;
+  p.n_qblocks = (Sq + tokens_per_cta - 1) / tokens_per_cta;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.causal = causal;
+  p.window = window;
+  p.lse = lse;
+  p.timeout_ns = kKernelTimeoutNs;
+
+  const long long grid = static_cast<long long>(p.n_qblocks) * B * Hkv * p.NP;
+  if (grid <= 0 || grid > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+
+  CUtensorMap tq, tk, tv, to;
+  const uint32_t tpt = 128 / p.Gp;
+  int rc;
+  if ((rc = encode_bf16_4d(&tq, q, D, Hq, Sq, B, p.Gp, tpt)) != FA_OK) return rc;
+  if ((rc = encode_bf16_4d(&tk, k, D, Hkv, Skv, B, 1, 128)) != FA_OK) return rc;
+  if ((rc = encode_bf16_4d(&tv, v, D, Hkv, Skv, B, 1, 128)) != FA_OK) return rc;
+  if ((rc = encode_bf16_4d(&to, o, D, Hq, Sq, B, p.Gp, tpt)) != FA_OK) return rc;
+
+  auto kernel = fa::fa_prefill_kernel<D>;
+  if ((rc = ensure_smem_attr(kernel, C::kSmemBytes,
+                             D == 128 ? g_attr_prefill128 : g_attr_prefill64)) != FA_OK)
+    return rc;
+  kernel<<<static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t decode_ws_layout(int B, int Hq, int D, int splits, size_t* lse_off) {
+  const size_t o_bytes = static_cast<size_t>(splits) * B * Hq * D * sizeof(float);
+  const size_t off = (o_bytes + 255) & ~size_t(255);
+  const size_t l_bytes = static_cast<size_t>(splits) * B * Hq * sizeof(float);
+  if (lse_off) *lse_off = off;
+  return (off + l_bytes + 255) & ~size_t(255);
+}
+
+template <int D>
+int launch_decode(const void* q, const int8_t* k, const int8_t* v, const float* ks, const float* vs,
+                  void* o, float* lse, int B, int Hq, int Hkv, int Skv, float scale, int splits,
+                  void* ws, cudaStream_t stream) {
+  size_t lse_off = 0;
+  decode_ws_layout(B, Hq, D, splits, &lse_off);
+  fa::DecodeParams p{};
+  p.q = static_cast<const uint16_t*>(q);
+  p.k = k;
+  p.v = v;
+  p.k_scale = ks;
+  p.v_scale = vs;
+  p.o_part = static_cast<float*>(ws);
+  p.lse_part = reinterpret_cast<float*>(static_cast<char*>(ws) + lse_off);
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Skv = Skv;
+  p.G = Hq / Hkv;
+  p.splits = splits;
+  p.chunk = (Skv + splits - 1) / splits;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  const long long gy = static_cast<long long>(B) * Hkv;
+  if (gy > 65535 || (p.G + 7) / 8 > 65535 || splits > 0x7fffffff) return FA_ERR_INVALID_ARG;
+  dim3 grid(splits, static_cast<unsigned>(gy), (p.G + 7) / 8);
+  fa::fa_decode_split_kernel<D><<<grid, 128, 0, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  fa::CombineParams cp{};
+  cp.o_part = p.o_part;
+  cp.lse_part = p.lse_part;
+  cp.o = static_cast<uint16_t*>(o);
+  cp.lse = lse;
+  cp.B = B;
+  cp.Hq = Hq;
+  cp.splits = splits;
+  fa::fa_decode_combine_kernel<D><<<B * Hq, D, 0, stream>>>(cp);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+__global__ void bounded_wait_selftest_kernel(uint64_t timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    fa::mbar_init(fa::smem_u32(&bar), 1);
+    fa::fence_mbar_init();
+    const fa::WaitCtl ctl{&abort_flag, timeout_ns};
+    // Nothing ever arrives on this barrier: the wait must give up on its own.
+    fa::mbar_wait(fa::smem_u32(&bar), 0, ctl);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+           int Sq, int Skv, int D, float scale, int causal, int window, void* stream) {
+  if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq <= 0 || Skv <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (window < 0 || (window > 0 && !causal)) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FA_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return D == 128 ? launch_prefill<128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, window, s)
+                  : launch_prefill<64>(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, window, s);
+}
+
+size_t fa_decode_int8_workspace_bytes(int B, int Hq, int D, int num_splits) {
+  if (B <= 0 || Hq <= 0 || D <= 0 || num_splits <= 0) return 0;
+  return decode_ws_layout(B, Hq, D, num_splits, nullptr);
+}
+
+int fa_decode_int8(const void* q, const int8_t* k, const int8_t* v, const float* k_scale,
+                   const float* v_scale, void* o, float* lse, int B, int Hq, int Hkv, int Skv,
+                   int D, float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+  if (!q || !k || !v || !k_scale || !v_scale || !o) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Skv <= 0 || D <= 0 || num_splits <= 0)
+    return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(k_scale) ||
+      !aligned16(v_scale) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FA_ERR_ALIGNMENT;
+  const size_t need = decode_ws_layout(B, Hq, D, num_splits, nullptr);
+  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return D == 128 ? launch_decode<128>(q, k, v, k_scale, v_scale, o, lse, B, Hq, Hkv, Skv, scale,
+                                       num_splits, workspace, s)
+                  : launch_decode<64>(q, k, v, k_scale, v_scale, o, lse, B, Hq, Hkv, Skv, scale,
+                                      num_splits, workspace, s);
+}
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: invalid argument";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: unsupported head dimension";
+    case FA_ERR_ALIGNMENT: return "FA_ERR_ALIGNMENT: pointer not 16-byte aligned";
+    case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: workspace missing or too small";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA call or kernel launch failed";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a kernel gave up a bounded wait";
+    default: return "unknown fa_status";
+  }
+}
+
+int fa_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  unsigned int v = 0;
+  if (cudaMemcpyFromSymbol(&v, fa::g_fa_device_status, sizeof v) != cudaSuccess) return FA_ERR_CUDA;
+  if (v == 0) return FA_OK;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(fa::g_fa_device_status, &zero, sizeof zero) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return (v & fa::kDevStatusTimeout) ? FA_ERR_TIMEOUT : FA_ERR_CUDA;
+}
+
+int fa_selftest_bounded_wait(int timeout_us, void* stream) {
+  if (timeout_us < 1 || timeout_us > 10000000) return FA_ERR_INVALID_ARG;
+  bounded_wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(timeout_us) * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // extern "C"

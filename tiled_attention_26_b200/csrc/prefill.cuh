@@ -1,0 +1,432 @@
+// Fused attention forward (prefill) for sm_100a.
+//
+// Computes O = softmax(Q K^T * scale + mask) V in one tiled pass with an online softmax, so
+// the score matrix never leaves the chip ("Flash Attention on Ascend: three techniques",
+// sections "tiling" and "online softmax"; "FlashAttention on Ascend NPUs", tiling section).
+//
+// One CTA owns 256 query rows, split into two 128-row tiles that share every K/V tile load.
+// Row r of the CTA is (token tok0 + r / Gp, query head h0 + r % Gp): Gp query heads of one KV
+// group are packed into the rows, so a K/V tile staged once in shared memory serves all of
+// them; the head mapping is that of an explicit repeat_interleave of the KV heads ("FlashAttention
+// variants: GQA, MQA, sparse attention", KV-expansion section) without ever building the copy.
+//
+// Warp roles (384 threads):
+//   warps 0-3  softmax for Q tile 0 (thread = row = TMEM lane), warps 4-7 the same for tile 1.
+//              Each reads its S row from TMEM, masks, updates the running max m and sum l,
+//              writes P (bf16) back into TMEM over S, rescales O in TMEM when m grew by more
+//              than 2^8, and at the end normalises O, stages it in shared memory and stores it
+//              with TMA, plus the row's log-sum-exp.
+//   warp 8     TMA producer: Q tiles once, then K_j, V_j into a ring of shared-memory stages.
+//   warp 9     allocates TMEM and issues tcgen05.mma from one thread:
+//                S_t = Q_t K_j^T (both operands in shared memory),
+//                O_t += P_t V_j  (P from TMEM, V from shared memory).
+//              Order per step: PV0(j), QK0(j+1), PV1(j), QK1(j+1), so that the tensor core
+//              works on one tile while the softmax warps work on the other.
+//   warps 10-11 idle.
+// TMEM columns: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D); P_t is the first
+// 64 columns of S_t (two bf16 per column).
+#pragma once
+
+#include "sm100.cuh"
+
+namespace fa {
+
+struct PrefillParams {
+  int B, Hq, Hkv, Sq, Skv;
+  int G;       // query heads per KV head
+  int Gp;      // query heads packed into the rows of one tile (power of two, divides G)
+  int NP;      // G / Gp
+  int n_qblocks;
+  float scale_log2;  // scale * log2(e)
+  int causal;
+  int window;  // <= 0: none
+  float* lse;  // [B, Hq, Sq] natural log, may be null
+  uint64_t timeout_ns;
+};
+
+template <int D>
+struct PrefillCfg {
+  static constexpr int kThreads = 384;
+  static constexpr int kHalves = D / 64;          // 128-byte swizzle atoms along D
+  static constexpr int kAtomBytes = 128 * 128;    // 128 rows x 128 bytes
+  static constexpr int kTileBytes = 128 * D * 2;  // one 128-row bf16 tile
+  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+  // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_final[2], drain
+  static constexpr int kBarQ = 0;
+  static constexpr int kBarKVFull = 1;
+  static constexpr int kBarKVEmpty = 1 + kStages;
+  static constexpr int kBarSFull = 1 + 2 * kStages;
+  static constexpr int kBarPFull = kBarSFull + 2;
+  static constexpr int kBarOFinal = kBarPFull + 2;
+  static constexpr int kBarDrain = kBarOFinal + 2;
+  static constexpr int kNumBars = kBarDrain + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + slack to align the base
+  static constexpr uint32_t kTmemCols = 512;
+  __device__ static constexpr uint32_t colS(int t) { return 128u * t; }
+  __device__ static constexpr uint32_t colO(int t) { return 256u + uint32_t(D) * t; }
+};
+
+// Visible keys of query token i: [vis_lo, vis_hi] (inclusive; empty when hi < lo).  Causal
+// masks are aligned to the bottom-right corner; a window keeps the W nearest keys, the
+// query's own position included ("FlashAttention variants: GQA, MQA, sparse attention",
+// sliding-window section).
+__device__ __forceinline__ int vis_lo(const PrefillParams& p, int i) {
+  return p.window > 0 ? max(0, i + (p.Skv - p.Sq) - p.window + 1) : 0;
+}
+__device__ __forceinline__ int vis_hi(const PrefillParams& p, int i) {
+  return p.causal ? min(i + (p.Skv - p.Sq), p.Skv - 1) : p.Skv - 1;
+}
+
+template <int D>
+__global__ void __launch_bounds__(384, 1)
+    fa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_k,
+                      const __grid_constant__ CUtensorMap tm_v,
+                      const __grid_constant__ CUtensorMap tm_o, const PrefillParams p) {
+  using C = PrefillCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + C::kQOff;
+  const uint32_t sKV = sbase + C::kKVOff;
+  auto bar = [&](int idx) { return sbase + C::kBarOff + 8u * idx; };
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  int* abort_flag = reinterpret_cast<int*>(smem + C::kMiscOff + 4);
+  const WaitCtl ctl{abort_flag, p.timeout_ns};
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work item: heaviest (last) query blocks first ----
+  const int per_qb = p.B * p.Hkv * p.NP;
+  const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x) / per_qb;
+  int rem = static_cast<int>(blockIdx.x) % per_qb;
+  const int b = rem / (p.Hkv * p.NP);
+  rem %= p.Hkv * p.NP;
+  const int g = rem / p.NP;
+  const int h0 = g * p.G + (rem % p.NP) * p.Gp;
+  const int tpt = 128 / p.Gp;  // tokens per tile
+  const int tok0 = qb * 2 * tpt;
+
+  // ---- key-tile range of each Q tile, and the rows that bound its masks ----
+  int jlo[2], jhi[2], lo_last[2], hi_first[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int first = tok0 + t * tpt;
+    const int last = min(first + tpt, p.Sq) - 1;
+    jlo[t] = jhi[t] = 0;
+    lo_last[t] = 0;
+    hi_first[t] = -1;
+    if (first < p.Sq) {
+      const int lo = vis_lo(p, first), hi = vis_hi(p, last);
+      lo_last[t] = vis_lo(p, last);
+      hi_first[t] = vis_hi(p, first);
+      if (hi >= lo && hi >= 0) {
+        jlo[t] = lo / 128;
+        jhi[t] = hi / 128 + 1;
+      }
+    }
+  }
+  const bool act0 = jhi[0] > jlo[0], act1 = jhi[1] > jlo[1];
+  const int J0 = act0 ? (act1 ? min(jlo[0], jlo[1]) : jlo[0]) : (act1 ? jlo[1] : 0);
+  const int J1 = act0 ? (act1 ? max(jhi[0], jhi[1]) : jhi[0]) : (act1 ? jhi[1] : 0);
+
+  // ---- setup ----
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kNumBars; ++i) {
+      uint32_t count = 1;
+      if (i == C::kBarPFull || i == C::kBarPFull + 1) count = 128;
+      mbar_init(bar(i), count);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_o);
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 8) {
+    // ================= TMA producer =================
+    if (lane == 0) {
+      int issued = 0;  // K/V copies started; slot of copy n is n % kStages
+      mbar_arrive_expect_tx(bar(C::kBarQ), 2 * C::kTileBytes);
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int hf = 0; hf < C::kHalves; ++hf)
+          tma_load_4d(sQ + t * C::kTileBytes + hf * C::kAtomBytes, &tm_q, bar(C::kBarQ), 64 * hf,
+                      h0, tok0 + t * tpt, b);
+      bool ok = true;
+      for (int j = J0; j < J1 && ok; ++j) {
+#pragma unroll
+        for (int kind = 0; kind < 2; ++kind) {
+          const int pos = 2 * (j - J0) + kind;
+          const int s = pos % C::kStages;
+          if (!mbar_wait(bar(C::kBarKVEmpty + s), ((pos / C::kStages) & 1) ^ 1, ctl)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(C::kBarKVFull + s), C::kTileBytes);
+#pragma unroll
+          for (int hf = 0; hf < C::kHalves; ++hf)
+            tma_load_4d(sKV + s * C::kTileBytes + hf * C::kAtomBytes, kind ? &tm_v : &tm_k,
+                        bar(C::kBarKVFull + s), 64 * hf, g, 128 * j, b);
+          issued = pos + 1;
+        }
+      }
+      // Every copy this thread started has landed before the CTA can exit (already true on
+      // the normal path; after a consumer gave up this waits, bounded, for copies in flight).
+      volatile int zero = 0;
+      const WaitCtl drain_ctl{&zero, p.timeout_ns};
+      mbar_wait(bar(C::kBarQ), 0, drain_ctl);
+      for (int s = 0; s < C::kStages && s < issued; ++s) {
+        const int last = s + C::kStages * ((issued - 1 - s) / C::kStages);
+        mbar_wait(bar(C::kBarKVFull + s), (last / C::kStages) & 1, drain_ctl);
+      }
+    }
+  } else if (warp == 9) {
+    // ================= MMA issuer =================
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
+      auto issue_qk = [&](int t, int slot) {
+        const uint32_t qa = sQ + t * C::kTileBytes, kb = sKV + slot * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * C::kAtomBytes + (kk % 4) * 32;
+          umma_ss(tmem + C::colS(t), smem_desc_sw128(qa + off, 16, 1024),
+                  smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int slot, bool first) {
+        const uint32_t vb = sKV + slot * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          umma_ts(tmem + C::colO(t), tmem + C::colS(t) + kk * 8,
+                  smem_desc_sw128(vb + kk * 16 * 128, C::kAtomBytes, 1024), idesc_pv,
+                  (first && kk == 0) ? 0u : 1u);
+        }
+      };
+      auto part = [&](int t, int j) { return j >= jlo[t] && j < jhi[t]; };
+      int n[2] = {0, 0};
+      bool ok = mbar_wait(bar(C::kBarQ), 0, ctl);
+      if (ok && J1 > J0) {
+        tc_fence_after();
+        ok = mbar_wait(bar(C::kBarKVFull + 0), 0, ctl);
+        if (ok) {
+          tc_fence_after();
+#pragma unroll
+          for (int t = 0; t < 2; ++t)
+            if (part(t, J0)) {
+              issue_qk(t, 0);
+              tc_commit(bar(C::kBarSFull + t));
+            }
+          tc_commit(bar(C::kBarKVEmpty + 0));
+        }
+        for (int j = J0; j < J1 && ok; ++j) {
+          const int vpos = 2 * (j - J0) + 1, vslot = vpos % C::kStages;
+          const int kpos = vpos + 1, kslot = kpos % C::kStages;
+          const bool nxt = j + 1 < J1;
+          if (!(ok = mbar_wait(bar(C::kBarKVFull + vslot), (vpos / C::kStages) & 1, ctl))) break;
+          tc_fence_after();
+          if (part(0, j)) {
+            if (!(ok = mbar_wait(bar(C::kBarPFull + 0), n[0] & 1, ctl))) break;
+            tc_fence_after();
+            issue_pv(0, vslot, j == jlo[0]);
+            ++n[0];
+            if (j == jhi[0] - 1) tc_commit(bar(C::kBarOFinal + 0));
+          }
+          if (nxt) {
+            if (!(ok = mbar_wait(bar(C::kBarKVFull + kslot), (kpos / C::kStages) & 1, ctl))) break;
+            tc_fence_after();
+            if (part(0, j + 1)) {
+              issue_qk(0, kslot);
+              tc_commit(bar(C::kBarSFull + 0));
+            }
+          }
+          if (part(1, j)) {
+            if (!(ok = mbar_wait(bar(C::kBarPFull + 1), n[1] & 1, ctl))) break;
+            tc_fence_after();
+            issue_pv(1, vslot, j == jlo[1]);
+            ++n[1];
+            if (j == jhi[1] - 1) tc_commit(bar(C::kBarOFinal + 1));
+          }
+          tc_commit(bar(C::kBarKVEmpty + vslot));
+          if (nxt) {
+            if (part(1, j + 1)) {
+              issue_qk(1, kslot);
+              tc_commit(bar(C::kBarSFull + 1));
+            }
+            tc_commit(bar(C::kBarKVEmpty + kslot));
+          }
+        }
+      }
+      // Drain: every MMA this thread issued has completed before TMEM is released.
+      tc_commit(bar(C::kBarDrain));
+      volatile int zero = 0;
+      const WaitCtl drain_ctl{&zero, p.timeout_ns};
+      mbar_wait(bar(C::kBarDrain), 0, drain_ctl);
+    }
+  } else if (warp < 8) {
+    // ================= softmax + correction + epilogue =================
+    const int t = warp >> 2;
+    const int r = threadIdx.x & 127;
+    const int t_jlo = t ? jlo[1] : jlo[0], t_jhi = t ? jhi[1] : jhi[0];
+    const int t_lo_last = t ? lo_last[1] : lo_last[0];
+    const int t_hi_first = t ? hi_first[1] : hi_first[0];
+    const uint32_t colS = t ? C::colS(1) : C::colS(0);
+    const uint32_t colO = t ? C::colO(1) : C::colO(0);
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+    const int R = t * 128 + r;
+    const int i = tok0 + R / p.Gp;
+    const int hh = h0 + R % p.Gp;
+    const int my_lo = vis_lo(p, i), my_hi = vis_hi(p, i);
+    const float sl2 = p.scale_log2;
+    float m = -INFINITY, l = 0.f;
+    int n = 0;
+    for (int j = t_jlo; j < t_jhi; ++j) {
+      bool ok = mbar_wait(bar(C::kBarSFull + t), n & 1, ctl);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      uint32_t sv[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(trow + colS + 32 * c, sv[c]);
+      tmem_wait_ld();
+      const bool need_mask = (128 * j < t_lo_last) || (128 * j + 127 > t_hi_first);
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const int key = 128 * j + 32 * c + k;
+            if (key < my_lo || key > my_hi) sv[c][k] = __float_as_uint(-INFINITY);
+          }
+      }
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int k = 0; k < 32; k += 4) {
+          mx0 = fmaxf(mx0, __uint_as_float(sv[c][k]));
+          mx1 = fmaxf(mx1, __uint_as_float(sv[c][k + 1]));
+          mx2 = fmaxf(mx2, __uint_as_float(sv[c][k + 2]));
+          mx3 = fmaxf(mx3, __uint_as_float(sv[c][k + 3]));
+        }
+      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      const float m_new = fmaxf(m, m_tile);
+      float alpha = 1.f;
+      bool resc = false;
+      if (n == 0) {
+        m = m_new;
+      } else if (m_new > m + 8.f) {
+        resc = true;
+        alpha = ex2(m - m_new);
+        m = m_new;
+      }
+      const float m_use = (m == -INFINITY) ? 0.f : m;
+      float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const int col = 64 * half + 2 * k;
+          const float a = ex2(fmaf(__uint_as_float(sv[col / 32][col % 32]), sl2, -m_use));
+          const float c2 = ex2(fmaf(__uint_as_float(sv[(col + 1) / 32][(col + 1) % 32]), sl2, -m_use));
+          s0 += a;
+          s1 += c2;
+          pk[k] = pack_bf16x2(a, c2);
+        }
+        tmem_st32(trow + colS + 32 * half, pk);
+      }
+      l = l * alpha + (s0 + s1);
+      tmem_wait_st();
+      if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t ov[32];
+          tmem_ld32(trow + colO + 32 * c, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
+          tmem_st32(trow + colO + 32 * c, ov);
+        }
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::kBarPFull + t));
+      ++n;
+    }
+
+    // ---- epilogue: O / l -> bf16 -> shared memory (swizzled like the O tensor map) -> TMA ----
+    bool have_o = false;
+    if (n > 0) {
+      bool ok = mbar_wait(bar(C::kBarOFinal + t), 0, ctl);
+      have_o = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+    }
+    const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+    const uint32_t stage = sQ + t * C::kTileBytes;  // Q tile t is no longer read
+    uint8_t* stage_ptr = smem + C::kQOff + t * C::kTileBytes;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t ov[32];
+      if (have_o) {
+        tmem_ld32(trow + colO + 32 * c, ov);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int k = 0; k < 32; ++k) ov[k] = 0u;
+      }
+      const int hf = c >> 1;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(ov[8 * q + 0]) * inv_l, __uint_as_float(ov[8 * q + 1]) * inv_l);
+        w.y = pack_bf16x2(__uint_as_float(ov[8 * q + 2]) * inv_l, __uint_as_float(ov[8 * q + 3]) * inv_l);
+        w.z = pack_bf16x2(__uint_as_float(ov[8 * q + 4]) * inv_l, __uint_as_float(ov[8 * q + 5]) * inv_l);
+        w.w = pack_bf16x2(__uint_as_float(ov[8 * q + 6]) * inv_l, __uint_as_float(ov[8 * q + 7]) * inv_l);
+        const int chunk = ((c & 1) * 4 + q) ^ (r & 7);
+        *reinterpret_cast<uint4*>(stage_ptr + hf * C::kAtomBytes + r * 128 + chunk * 16) = w;
+      }
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(1 + t, 128);
+    if (r == 0 && tok0 + t * tpt < p.Sq) {
+#pragma unroll
+      for (int hf = 0; hf < C::kHalves; ++hf)
+        tma_store_4d(&tm_o, stage + hf * C::kAtomBytes, 64 * hf, h0, tok0 + t * tpt, b);
+      tma_store_commit();
+      tma_store_wait_read_all();
+    }
+    if (p.lse != nullptr && i < p.Sq) {
+      const float lse = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+      p.lse[(static_cast<size_t>(b) * p.Hq + hh) * p.Sq + i] = lse;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace fa
