@@ -1,0 +1,420 @@
+#!/usr/bin/env python
+"""Benchmark of the fused attention hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+  * prefill  (fa_fwd): MHA, B=2, Hq=Hkv=32, S=4096, D=128, causal, bf16 -- the workload the
+    headline metric is quoted on (attention forward TFLOP/s);
+  * decode   (fa_decode_int8, split kernel + combine kernel): B=16, Hq=32, Hkv=8, Skv=32768,
+    D=128, INT8 KV cache with per-token scales, 16 splits (KV-read GB/s).
+Inputs are seeded synthetic N(0,1) draws (see synthetic.py) resident in HBM; both inputs are
+larger than the 126 MB L2 (prefill 268 MB, decode 1.1 GB), so no flush is needed between steps.
+
+Prints ONE JSON line (rank 0).  Under torchrun every rank runs the same workload on its own
+GPU with its own seeds (independent problems, weak scaling, no data-path collective); times are
+CUDA-event times, max over ranks.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded row sample of the same prefill
+workload instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attn fwd TFLOP/s & % bf16 TC peak; decode KV-read GB/s & % HBM peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# dram__bytes_read.sum + dram__bytes_write.sum per launch from ncu, keyed by the sha256 of the
+# kernel sources they were taken on; a kernel edited since then reports traffic = null.
+NCU_TRAFFIC = {
+    "prefill": {},
+    "decode": {},
+}
+
+
+def source_hash(*names):
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "tiled_attention_26_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def prefill_flops(w) -> int:
+    """Algorithmic flops: 4*D per visible (query, key) pair (QK^T and PV, 2 flops per MAC)."""
+    pairs = 0
+    off = w.Skv - w.Sq
+    for i in range(w.Sq):
+        hi = min(i + off, w.Skv - 1) if w.causal else w.Skv - 1
+        lo = max(0, i + off - w.window + 1) if w.window > 0 else 0
+        pairs += max(0, hi - lo + 1)
+    return pairs * 4 * w.D * w.B * w.Hq
+
+
+def decode_bytes(w) -> int:
+    """Algorithmic bytes: int8 K and V, fp32 scales, bf16 q in and o out, fp32 LSE."""
+    kv = 2 * w.B * w.Skv * w.Hkv * w.D
+    scales = 2 * w.B * w.Hkv * w.Skv * 4
+    qo = 2 * w.B * w.Hq * w.D * 2
+    return kv + scales + qo + w.B * w.Hq * 4
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 100 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"samples": 0, "sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(n)
+        return {"samples": len(sm), "sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
+
+
+class OracleTimer:
+    """Times the fp64 oracle, as it stands, on bounded row samples of the prefill workload."""
+
+    def __init__(self, w):
+        import numpy as np
+
+        import oracle
+        import synthetic
+
+        self.w, self.oracle, self.np, self.synthetic = w, oracle, np, synthetic
+        self.q, self.k, self.v = synthetic.make_qkv(w)
+        self.cores = oracle.max_threads()
+        t0 = time.perf_counter()
+        self.run(self.rows(w.seed(39), 64))
+        self.rows_per_s = 64 / max(time.perf_counter() - t0, 1e-3)
+
+    def rows(self, seed, n):
+        np, w = self.np, self.w
+        raw = self.synthetic.splitmix64(seed, 0, 3 * n).reshape(-1, 3)
+        return np.stack([raw[:, 0] % np.uint64(w.B), raw[:, 1] % np.uint64(w.Hq),
+                         raw[:, 2] % np.uint64(w.Sq)], axis=1).astype(np.int64)
+
+    def flops(self, rows):
+        w = self.w
+        off = w.Skv - w.Sq
+        n = 0
+        for _, _, i in rows:
+            hi = min(i + off, w.Skv - 1) if w.causal else w.Skv - 1
+            lo = max(0, i + off - w.window + 1) if w.window > 0 else 0
+            n += 4 * w.D * max(0, hi - lo + 1)
+        return n
+
+    def run(self, rows):
+        w = self.w
+        self.oracle.attn_rows(self.q, self.k, self.v, w.scale, w.causal, w.window, rows)
+
+    def sample(self, seed, budget_s):
+        """Returns (flops, seconds, n_rows) for a sample sized to take about budget_s."""
+        n = max(8, int(self.rows_per_s * budget_s))
+        rows = self.rows(seed, n)
+        t0 = time.perf_counter()
+        self.run(rows)
+        return self.flops(rows), time.perf_counter() - t0, n
+
+
+def cpu_baseline(w, budget_s: float, seed: int):
+    t = OracleTimer(w)
+    fl, dt, n = t.sample(seed, budget_s)
+    return {"value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": t.cores, "kind": "oracle",
+            "sample": f"{n} seeded (b, h, i) rows of the prefill workload, every visible key, "
+                      f"fp64, {dt:.1f} s"}, dt
+
+
+def run_reference(args):
+    import synthetic
+
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    w = synthetic.WORKLOADS["mha_causal"]
+    timer = OracleTimer(w)
+    per_step = min(4.0, 120.0 / max(1, args.steps + args.warmup))
+    tot_f, tot_t, n_rows = 0, 0.0, 0
+    for step in range(args.warmup + args.steps):
+        fl, dt, n = timer.sample(w.seed(50 + step), per_step)
+        if step >= args.warmup:
+            tot_f, tot_t, n_rows = tot_f + fl, tot_t + dt, n_rows + n
+    value = tot_f / tot_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * tot_t / max(1, args.steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "mha_causal prefill B=2 Hq=Hkv=32 S=4096 D=128 causal "
+                               "(bounded row sample per step)", "parallelism": "rank 0 only"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": timer.cores, "kind": "oracle",
+                         "sample": f"{n_rows} seeded (b, h, i) rows over {args.steps} steps, every "
+                                   f"visible key, fp64, {tot_t:.1f} s"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+
+    import synthetic
+    import tiled_attention_26_b200 as fa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    wp = synthetic.WORKLOADS["mha_causal"]
+    wd = synthetic.WORKLOADS["decode_int8"]
+    dev = torch.device("cuda", local)
+    seed_off = 1000 * rank
+    q = synthetic.normal_bf16_torch(wp.seed(0) + seed_off, wp.q_shape(), dev)
+    k = synthetic.normal_bf16_torch(wp.seed(1) + seed_off, wp.kv_shape(), dev)
+    v = synthetic.normal_bf16_torch(wp.seed(2) + seed_off, wp.kv_shape(), dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((wp.B, wp.Hq, wp.Sq), dtype=torch.float32, device=dev)
+    dq = synthetic.normal_bf16_torch(wd.seed(0) + seed_off, wd.q_shape(), dev)
+    dk, dks = synthetic.quantize_int8_per_token_torch(
+        synthetic.normal_bf16_torch(wd.seed(1) + seed_off, wd.kv_shape(), dev))
+    dv, dvs = synthetic.quantize_int8_per_token_torch(
+        synthetic.normal_bf16_torch(wd.seed(2) + seed_off, wd.kv_shape(), dev))
+    do = torch.empty_like(dq)
+    dlse = torch.empty((wd.B, wd.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(fa.fa_decode_int8_workspace_bytes(wd.B, wd.Hq, wd.D, wd.num_splits),
+                     dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+
+    def prefill():
+        fa.fa_fwd(q, k, v, causal=True, scale=wp.scale, o=o, lse=lse, stream=stream)
+
+    def decode():
+        fa.fa_decode_int8(dq, dk, dv, dks, dvs, num_splits=wd.num_splits, scale=wd.scale, o=do,
+                          lse=dlse, workspace=ws, stream=stream)
+
+    for _ in range(args.warmup):
+        prefill()
+        decode()
+    torch.cuda.synchronize()
+    if fa.fa_device_status() != 0:
+        raise RuntimeError("a kernel reported a device-side timeout during warm-up")
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    visible = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
+    phys = int(visible[local]) if local < len(visible) and visible[local].strip().isdigit() else local
+    clocks = ClockSampler(phys)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.25)  # let the sampler start before the timed region
+    start.record(stream)
+    for s in range(K):
+        ev[s][0].record(stream)
+        prefill()
+        ev[s][1].record(stream)
+        decode()
+        ev[s][2].record(stream)
+    stop.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    if fa.fa_device_status() != 0:
+        raise RuntimeError("a kernel reported a device-side timeout in the timed region")
+
+    total_ms = max_over_ranks(start.elapsed_time(stop))
+    pre_ms = [ev[s][0].elapsed_time(ev[s][1]) for s in range(K)]
+    dec_ms = [ev[s][1].elapsed_time(ev[s][2]) for s in range(K)]
+    pre_sum = max_over_ranks(sum(pre_ms))
+    dec_sum = max_over_ranks(sum(dec_ms))
+
+    flops = prefill_flops(wp)
+    dbytes = decode_bytes(wd)
+    peaks, peak_src = load_peaks()
+    pre_tflops = world * K * flops / (pre_sum * 1e-3) / 1e12
+    dec_gbs = world * K * dbytes / (dec_sum * 1e-3) / 1e9
+    pre_avg_s = sum(pre_ms) / K * 1e-3
+    dec_avg_s = sum(dec_ms) / K * 1e-3
+    achieved = flops / pre_avg_s / 1e12
+    d_achieved = dbytes / dec_avg_s / 1e9
+
+    # ---- end to end through the public API, host buffers, copies inside the timed region ----
+    e2e = None
+    if args.e2e_steps > 0:
+        hq, hk, hv = (t.cpu().pin_memory() for t in (q, k, v))
+        ho, hl = torch.empty_like(hq).pin_memory(), lse.cpu().pin_memory()
+        hdq, hdk, hdv, hdks, hdvs = (t.cpu().pin_memory() for t in (dq, dk, dv, dks, dvs))
+        hdo, hdl = torch.empty_like(hdq).pin_memory(), dlse.cpu().pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdq, hdk, hdv, hdks, hdvs))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hl, hdo, hdl))
+        E = args.e2e_steps
+        e3 = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(E)]
+        barrier()
+        torch.cuda.synchronize()
+        for s in range(E):
+            e3[s][0].record(stream)
+            for d_, h_ in ((q, hq), (k, hk), (v, hv)):
+                d_.copy_(h_, non_blocking=True)
+            prefill()
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+            e3[s][1].record(stream)
+            for d_, h_ in ((dq, hdq), (dk, hdk), (dv, hdv), (dks, hdks), (dvs, hdvs)):
+                d_.copy_(h_, non_blocking=True)
+            decode()
+            hdo.copy_(do, non_blocking=True)
+            hdl.copy_(dlse, non_blocking=True)
+            e3[s][2].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        p_ms = max_over_ranks(sum(e3[s][0].elapsed_time(e3[s][1]) for s in range(E)))
+        d_ms = max_over_ranks(sum(e3[s][1].elapsed_time(e3[s][2]) for s in range(E)))
+        e2e = {"value": world * E * flops / (p_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": E,
+               "decode": {"value": world * E * dbytes / (d_ms * 1e-3) / 1e9, "unit": "GB/s"},
+               "ms_per_step": (p_ms + d_ms) / E}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu, _ = cpu_baseline(wp, args.cpu_budget, seed=wp.seed(40))
+
+    if rank == 0:
+        tp = NCU_TRAFFIC["prefill"].get(source_hash("prefill.cuh", "sm100.cuh"))
+        td = NCU_TRAFFIC["decode"].get(source_hash("decode.cuh", "sm100.cuh"))
+        line = {
+            "metric": METRIC,
+            "value": pre_tflops,
+            "unit": "TFLOP/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": total_ms / K,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic",
+            "config": {
+                "workload": "one step = mha_causal prefill (B=2, Hq=Hkv=32, S=4096, D=128, causal, "
+                            "bf16) + decode_int8 (B=16, Hq=32, Hkv=8, Skv=32768, D=128, INT8 KV, "
+                            "16 splits)",
+                "prefill_flops_per_step": flops,
+                "decode_bytes_per_step": dbytes,
+                "l2": "no flush: every step reads inputs larger than L2 (prefill 268 MB, decode 1.1 GB)",
+                "parallelism": f"{world} independent GPU(s), no data-path collective",
+            },
+            "decode": {"value": dec_gbs, "unit": "GB/s", "frac_of_hbm": dec_gbs / world / peaks["hbm_gbs"],
+                       "ms_per_call": dec_sum / K},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                         "traffic": tp, "kernel": "fa_prefill_kernel<128>",
+                         "peak_source": f"{peak_src} bf16 dense (burst)",
+                         "ms_per_launch": pre_avg_s * 1e3},
+            "roofline_decode": {"bound": "hbm", "achieved": d_achieved, "peak": peaks["hbm_gbs"],
+                                "unit": "GB/s", "frac": d_achieved / peaks["hbm_gbs"],
+                                "traffic": td,
+                                "kernel": "fa_decode_split_kernel<128> + fa_decode_combine_kernel<128>",
+                                "peak_source": f"{peak_src} copy bandwidth",
+                                "ms_per_call": dec_avg_s * 1e3},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 3 * K,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
