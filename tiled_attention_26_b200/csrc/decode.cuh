@@ -65,12 +65,6 @@ __device__ __forceinline__ uint2 ldg_stream8(const void* p) {
   return r;
 }
 
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
-}
-
 // Two biased bytes (x + 128) in the low bytes of a fp16 pair with exponent 2^10 give
 // 1024 + x + 128 exactly; subtracting 1152 leaves x exactly.
 constexpr uint32_t kMagic64 = 0x64646464u;

@@ -107,6 +107,16 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
   if ((rc = ensure_smem_attr(kernel, C::kSmemBytes,
                              D == 128 ? g_attr_prefill128 : g_attr_prefill64)) != FA_OK)
     return rc;
+  // The kernel redistributes its launch registers between warpgroups (setmaxnreg); that only
+  // completes if the launch gave every thread at least kMinLaunchRegs.
+  static int launch_regs[2] = {-1, -1};
+  int& regs = launch_regs[D == 128 ? 1 : 0];
+  if (regs < 0) {
+    cudaFuncAttributes attr;
+    if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return FA_ERR_CUDA;
+    regs = attr.numRegs;
+  }
+  if (regs < C::kMinLaunchRegs) return FA_ERR_UNSUPPORTED;
   kernel<<<static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }

@@ -19,7 +19,7 @@
 //   warp 8     TMA producer: Q tiles once, then K_j, V_j into a ring of shared-memory stages.
 //   warp 9     allocates TMEM and issues tcgen05.mma from one thread:
 //                S_t = Q_t K_j^T (both operands in shared memory),
-//                O_t += P_t V_j  (P from TMEM, V from shared memory).
+//                O_t += P_t V_j  (P from TMEM, V from shared memory; P arrives in two halves).
 //              Order per step: PV0(j), QK0(j+1), PV1(j), QK1(j+1), so that the tensor core
 //              works on one tile while the softmax warps work on the other.
 //   warps 10-11 idle.
@@ -30,6 +30,10 @@
 #include "sm100.cuh"
 
 namespace fa {
+
+#ifndef FA_REGS_SOFTMAX
+#define FA_REGS_SOFTMAX 216
+#endif
 
 struct PrefillParams {
   int B, Hq, Hkv, Sq, Skv;
@@ -50,22 +54,31 @@ struct PrefillCfg {
   static constexpr int kHalves = D / 64;          // 128-byte swizzle atoms along D
   static constexpr int kAtomBytes = 128 * 128;    // 128 rows x 128 bytes
   static constexpr int kTileBytes = 128 * D * 2;  // one 128-row bf16 tile
-  static constexpr int kStages = (D == 128) ? 4 : 8;
+#ifndef FA_KV_STAGES_D128
+#define FA_KV_STAGES_D128 4
+#endif
+  static constexpr int kStages = (D == 128) ? FA_KV_STAGES_D128 : 8;
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
-  // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_final[2], drain
+  // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2 tiles][2 halves],
+  // o_final[2], drain
   static constexpr int kBarQ = 0;
   static constexpr int kBarKVFull = 1;
   static constexpr int kBarKVEmpty = 1 + kStages;
   static constexpr int kBarSFull = 1 + 2 * kStages;
   static constexpr int kBarPFull = kBarSFull + 2;
-  static constexpr int kBarOFinal = kBarPFull + 2;
+  static constexpr int kBarOFinal = kBarPFull + 4;
   static constexpr int kBarDrain = kBarOFinal + 2;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + slack to align the base
   static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kRegsSoftmax = FA_REGS_SOFTMAX;
+  // the rest of the 384 x 168 launch registers go to the producer / MMA warpgroup
+  static constexpr uint32_t kRegsOther = ((168 * 384 - 2 * 128 * kRegsSoftmax) / 128) / 8 * 8;
+  static constexpr int kMinLaunchRegs =
+      (2 * 128 * kRegsSoftmax + 128 * kRegsOther + kThreads - 1) / kThreads;
   __device__ static constexpr uint32_t colS(int t) { return 128u * t; }
   __device__ static constexpr uint32_t colO(int t) { return 256u + uint32_t(D) * t; }
 };
@@ -79,6 +92,68 @@ __device__ __forceinline__ int vis_lo(const PrefillParams& p, int i) {
 }
 __device__ __forceinline__ int vis_hi(const PrefillParams& p, int i) {
   return p.causal ? min(i + (p.Skv - p.Sq), p.Skv - 1) : p.Skv - 1;
+}
+
+#ifndef FA_EXP2_EMU_OF8
+#define FA_EXP2_EMU_OF8 0  // of every 8 column pairs, this many use exp2_fma on unmasked tiles
+#endif
+constexpr int kEmuOf8 = FA_EXP2_EMU_OF8;
+#ifndef FA_PACK_INT
+#define FA_PACK_INT 0  // 1: bf16 rounding with an integer add and a byte permute instead of cvt
+#endif
+
+// Two non-negative fp32 values -> bf16x2 (lo in the low half).
+__device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
+#if FA_PACK_INT
+  // round half up on the magnitude (the values are >= 0), keep the upper halves
+  return prmt(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632u);
+#else
+  return pack_bf16x2(lo, hi);
+#endif
+}
+
+// Row maximum of the 128 raw scores (3-input max, 8 independent chains).
+__device__ __forceinline__ float row_max128(const uint32_t (&sv)[4][32]) {
+  float m[8];
+#pragma unroll
+  for (int c = 0; c < 8; ++c) m[c] = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const int col = 16 * i + 2 * c;
+      m[c] = fmax3(m[c], __uint_as_float(sv[col / 32][col % 32]),
+                   __uint_as_float(sv[(col + 1) / 32][(col + 1) % 32]));
+    }
+  return fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+}
+
+// p = 2^(s * sl2 - m_use) for the 64 columns of one half, written to TMEM as 32 bf16 pairs;
+// returns the fp32 sum of the half through acc (two packed partial sums).
+template <bool kEmu>
+__device__ __forceinline__ void exp_half(const uint32_t (&sv)[4][32], int half, float sl2,
+                                         float m_use, uint32_t taddr, uint64_t& acc0,
+                                         uint64_t& acc1) {
+  const uint64_t scale2 = f2(sl2, sl2), negm2 = f2(-m_use, -m_use);
+  uint32_t pk[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const int col = 64 * half + 2 * k;
+    const uint64_t x = f2_fma(f2(__uint_as_float(sv[col / 32][col % 32]),
+                                 __uint_as_float(sv[(col + 1) / 32][(col + 1) % 32])),
+                              scale2, negm2);
+    float x0, x1, a, c;
+    f2_split(x, x0, x1);
+    if (kEmu && (k % 8) < kEmuOf8) {
+      exp2_fma_x2(x0, x1, a, c);
+    } else {
+      a = ex2(x0);
+      c = ex2(x1);
+    }
+    if (k & 1) acc1 = f2_add(acc1, f2(a, c)); else acc0 = f2_add(acc0, f2(a, c));
+    pk[k] = pack_p(a, c);
+  }
+  tmem_st32(taddr + 32 * half, pk);
 }
 
 template <int D>
@@ -139,7 +214,7 @@ __global__ void __launch_bounds__(384, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kNumBars; ++i) {
       uint32_t count = 1;
-      if (i == C::kBarPFull || i == C::kBarPFull + 1) count = 128;
+      if (i >= C::kBarPFull && i < C::kBarPFull + 4) count = 128;
       mbar_init(bar(i), count);
     }
     *abort_flag = 0;
@@ -160,6 +235,11 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
+  // Registers: the softmax warpgroups hold a full S row (128 fp32) per thread; the producer /
+  // MMA warpgroup needs few.  2*128*216 + 128*56 = 62464 <= 384 threads * 168 at launch (the
+  // host refuses to launch if the kernel was given fewer than kMinLaunchRegs per thread).
+  if (warp >= 8) {
+    setmaxnreg_dec<C::kRegsOther>();
   if (warp == 8) {
     // ================= TMA producer =================
     if (lane == 0) {
@@ -201,6 +281,8 @@ __global__ void __launch_bounds__(384, 1)
     }
   } else if (warp == 9) {
     // ================= MMA issuer =================
+    // One thread issues both Q tiles' chains in the order PV0(j), QK0(j+1), PV1(j), QK1(j+1):
+    // the tensor core finishes one tile's S while the softmax warps work on the other tile.
     if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, true);
@@ -213,23 +295,39 @@ __global__ void __launch_bounds__(384, 1)
                   smem_desc_sw128(kb + off, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, int slot, bool first) {
+      // O_t += P_t V over keys [64 * half, 64 * half + 64) of the tile
+      auto issue_pv_half = [&](int t, int slot, int half, bool first) {
         const uint32_t vb = sKV + slot * C::kTileBytes;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int kk = 4 * half + k4;
           umma_ts(tmem + C::colO(t), tmem + C::colS(t) + kk * 8,
                   smem_desc_sw128(vb + kk * 16 * 128, C::kAtomBytes, 1024), idesc_pv,
                   (first && kk == 0) ? 0u : 1u);
         }
+      };
+      // P_t arrives in two halves; the first half of PV starts while the softmax warps are
+      // still computing the second.
+      auto issue_pv = [&](int t, int slot, bool first, int phase) -> bool {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          if (!mbar_wait(bar(C::kBarPFull + 2 * t + half), phase, ctl)) return false;
+          tc_fence_after();
+          issue_pv_half(t, slot, half, first);
+        }
+        return true;
+      };
+      auto kv_wait = [&](int pos) {
+        const bool ok = mbar_wait(bar(C::kBarKVFull + pos % C::kStages), (pos / C::kStages) & 1, ctl);
+        tc_fence_after();
+        return ok;
       };
       auto part = [&](int t, int j) { return j >= jlo[t] && j < jhi[t]; };
       int n[2] = {0, 0};
       bool ok = mbar_wait(bar(C::kBarQ), 0, ctl);
       if (ok && J1 > J0) {
         tc_fence_after();
-        ok = mbar_wait(bar(C::kBarKVFull + 0), 0, ctl);
-        if (ok) {
-          tc_fence_after();
+        if ((ok = kv_wait(0))) {
 #pragma unroll
           for (int t = 0; t < 2; ++t)
             if (part(t, J0)) {
@@ -239,30 +337,24 @@ __global__ void __launch_bounds__(384, 1)
           tc_commit(bar(C::kBarKVEmpty + 0));
         }
         for (int j = J0; j < J1 && ok; ++j) {
-          const int vpos = 2 * (j - J0) + 1, vslot = vpos % C::kStages;
-          const int kpos = vpos + 1, kslot = kpos % C::kStages;
+          const int vpos = 2 * (j - J0) + 1, kpos = vpos + 1;
+          const int vslot = vpos % C::kStages, kslot = kpos % C::kStages;
           const bool nxt = j + 1 < J1;
-          if (!(ok = mbar_wait(bar(C::kBarKVFull + vslot), (vpos / C::kStages) & 1, ctl))) break;
-          tc_fence_after();
+          if (!(ok = kv_wait(vpos))) break;
           if (part(0, j)) {
-            if (!(ok = mbar_wait(bar(C::kBarPFull + 0), n[0] & 1, ctl))) break;
-            tc_fence_after();
-            issue_pv(0, vslot, j == jlo[0]);
+            if (!(ok = issue_pv(0, vslot, j == jlo[0], n[0] & 1))) break;
             ++n[0];
             if (j == jhi[0] - 1) tc_commit(bar(C::kBarOFinal + 0));
           }
           if (nxt) {
-            if (!(ok = mbar_wait(bar(C::kBarKVFull + kslot), (kpos / C::kStages) & 1, ctl))) break;
-            tc_fence_after();
+            if (!(ok = kv_wait(kpos))) break;
             if (part(0, j + 1)) {
               issue_qk(0, kslot);
               tc_commit(bar(C::kBarSFull + 0));
             }
           }
           if (part(1, j)) {
-            if (!(ok = mbar_wait(bar(C::kBarPFull + 1), n[1] & 1, ctl))) break;
-            tc_fence_after();
-            issue_pv(1, vslot, j == jlo[1]);
+            if (!(ok = issue_pv(1, vslot, j == jlo[1], n[1] & 1))) break;
             ++n[1];
             if (j == jhi[1] - 1) tc_commit(bar(C::kBarOFinal + 1));
           }
@@ -282,7 +374,9 @@ __global__ void __launch_bounds__(384, 1)
       const WaitCtl drain_ctl{&zero, p.timeout_ns};
       mbar_wait(bar(C::kBarDrain), 0, drain_ctl);
     }
-  } else if (warp < 8) {
+  }  // warps 10-11 have no role
+  } else {
+    setmaxnreg_inc<C::kRegsSoftmax>();
     // ================= softmax + correction + epilogue =================
     const int t = warp >> 2;
     const int r = threadIdx.x & 127;
@@ -317,17 +411,7 @@ __global__ void __launch_bounds__(384, 1)
             if (key < my_lo || key > my_hi) sv[c][k] = __float_as_uint(-INFINITY);
           }
       }
-      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int k = 0; k < 32; k += 4) {
-          mx0 = fmaxf(mx0, __uint_as_float(sv[c][k]));
-          mx1 = fmaxf(mx1, __uint_as_float(sv[c][k + 1]));
-          mx2 = fmaxf(mx2, __uint_as_float(sv[c][k + 2]));
-          mx3 = fmaxf(mx3, __uint_as_float(sv[c][k + 3]));
-        }
-      const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
+      const float m_tile = row_max128(sv) * sl2;
       const float m_new = fmaxf(m, m_tile);
       float alpha = 1.f;
       bool resc = false;
@@ -338,24 +422,9 @@ __global__ void __launch_bounds__(384, 1)
         alpha = ex2(m - m_new);
         m = m_new;
       }
-      const float m_use = (m == -INFINITY) ? 0.f : m;
-      float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const int col = 64 * half + 2 * k;
-          const float a = ex2(fmaf(__uint_as_float(sv[col / 32][col % 32]), sl2, -m_use));
-          const float c2 = ex2(fmaf(__uint_as_float(sv[(col + 1) / 32][(col + 1) % 32]), sl2, -m_use));
-          s0 += a;
-          s1 += c2;
-          pk[k] = pack_bf16x2(a, c2);
-        }
-        tmem_st32(trow + colS + 32 * half, pk);
-      }
-      l = l * alpha + (s0 + s1);
-      tmem_wait_st();
+      // Lazy correction: O (accumulated up to the previous tile, complete since S of this tile
+      // is) is rescaled only when the running max grew by more than 2^8; otherwise the stale max
+      // stays the reference and p may reach 2^8, which fp32 O and l absorb exactly.
       if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
@@ -366,10 +435,28 @@ __global__ void __launch_bounds__(384, 1)
           for (int k = 0; k < 32; ++k) ov[k] = __float_as_uint(__uint_as_float(ov[k]) * alpha);
           tmem_st32(trow + colO + 32 * c, ov);
         }
-        tmem_wait_st();
       }
-      tc_fence_before();
-      mbar_arrive(bar(C::kBarPFull + t));
+      const float m_use = (m == -INFINITY) ? 0.f : m;
+      // p = 2^(s * scale * log2(e) - m) as bf16 pairs over the S columns, one half at a time;
+      // each half is released to the MMA warp as soon as it is in TMEM.  Unmasked tiles take
+      // kEmuOf8 of every 8 pairs through exp2_fma (FMA pipe) to offload the MUFU pipe; masked
+      // tiles use MUFU only, so masked scores give exactly 0.
+      uint64_t acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        if (need_mask) {
+          exp_half<false>(sv, half, sl2, m_use, trow + colS, acc0, acc1);
+        } else {
+          exp_half<true>(sv, half, sl2, m_use, trow + colS, acc0, acc1);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(C::kBarPFull + 2 * t + half));
+      }
+      float a0, a1, a2, a3;
+      f2_split(acc0, a0, a1);
+      f2_split(acc1, a2, a3);
+      l = l * alpha + ((a0 + a1) + (a2 + a3));
       ++n;
     }
 
