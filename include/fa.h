@@ -106,6 +106,37 @@ FA_API int fa_decode_int8(const void* q, const int8_t* k, const int8_t* v, const
                    int D, float scale, int num_splits, void* workspace, size_t workspace_bytes,
                    void* stream);
 
+/*
+ * Allocation-free variant of fa_decode_int8 (the pages have no counterpart; this is a calling
+ * convenience of this library).
+ *
+ * Who needs it: callers that cannot call cudaMalloc at the point where they decode -- code
+ * running under a memory manager that owns the whole device budget and forbids allocations it
+ * did not make, latency-critical loops where an allocation's implicit device synchronisation is
+ * not acceptable, and plain C callers without an allocator of their own.  They pass inputs and
+ * outputs exactly as for fa_decode_int8 but no workspace.
+ *
+ * Scratch: the split partials live in a fixed array inside the library, of
+ * FA_DECODE_INT8_NOALLOC_MAX_SCRATCH bytes per GPU, which every GPU that loads the library holds
+ * until the process exits.  Calls whose fa_decode_int8_workspace_bytes(B, Hq, D, num_splits)
+ * exceeds that size return FA_ERR_WORKSPACE and launch nothing.  This function calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current and caches it; make that first call before any stream capture.
+ *
+ * Every call on a GPU shares the one array, and the array keeps the last call's contents (the
+ * kernels overwrite every byte they read, so nothing needs clearing).  Calls whose kernels can
+ * overlap on the GPU -- on different streams, or from different host threads -- race on it;
+ * order such calls on one stream or use fa_decode_int8 with separate workspaces.
+ * Arguments, layouts and status codes are otherwise those of fa_decode_int8.
+ */
+#define FA_DECODE_INT8_NOALLOC_MAX_SCRATCH (8u << 20)
+FA_API int fa_decode_int8_noalloc(const void* q, const int8_t* k, const int8_t* v,
+                                  const float* k_scale, const float* v_scale, void* o, float* lse,
+                                  int B, int Hq, int Hkv, int Skv, int D, float scale,
+                                  int num_splits, void* stream);
+
 /* Static, human-readable name of a status code.  Never NULL. */
 FA_API const char* fa_status_string(int status);
 

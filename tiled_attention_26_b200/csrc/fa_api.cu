@@ -14,6 +14,10 @@
 #include "prefill.cuh"
 #include "sm100.cuh"
 
+// Scratch of the allocation-free decode entry point: one copy per GPU that loads the library,
+// held until the process exits.  Shared by every call of fa_decode_int8_noalloc on that GPU.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FA_DECODE_INT8_NOALLOC_MAX_SCRATCH];
+
 namespace {
 
 constexpr uint64_t kKernelTimeoutNs = 4000000000ull;  // bounded waits give up after 4 s
@@ -168,6 +172,25 @@ int launch_decode(const void* q, const int8_t* k, const int8_t* v, const float* 
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// Device address of g_noalloc_scratch on the current device.  In host code the symbol name is
+// only a host-side stand-in, so the address is looked up once per device, with that device
+// current, and cached.
+int noalloc_scratch_address(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return FA_ERR_CUDA;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return FA_OK;
+}
+
 __global__ void bounded_wait_selftest_kernel(uint64_t timeout_ns) {
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;
@@ -252,6 +275,30 @@ int fa_device_status(void* stream) {
   if (cudaMemcpyToSymbol(fa::g_fa_device_status, &zero, sizeof zero) != cudaSuccess)
     return FA_ERR_CUDA;
   return (v & fa::kDevStatusTimeout) ? FA_ERR_TIMEOUT : FA_ERR_CUDA;
+}
+
+int fa_decode_int8_noalloc(const void* q, const int8_t* k, const int8_t* v, const float* k_scale,
+                           const float* v_scale, void* o, float* lse, int B, int Hq, int Hkv,
+                           int Skv, int D, float scale, int num_splits, void* stream) {
+  if (!q || !k || !v || !k_scale || !v_scale || !o) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Skv <= 0 || D <= 0 || num_splits <= 0)
+    return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(k_scale) ||
+      !aligned16(v_scale) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FA_ERR_ALIGNMENT;
+  if (decode_ws_layout(B, Hq, D, num_splits, nullptr) > FA_DECODE_INT8_NOALLOC_MAX_SCRATCH)
+    return FA_ERR_WORKSPACE;
+  void* ws = nullptr;
+  const int rc = noalloc_scratch_address(&ws);
+  if (rc != FA_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return D == 128 ? launch_decode<128>(q, k, v, k_scale, v_scale, o, lse, B, Hq, Hkv, Skv, scale,
+                                       num_splits, ws, s)
+                  : launch_decode<64>(q, k, v, k_scale, v_scale, o, lse, B, Hq, Hkv, Skv, scale,
+                                      num_splits, ws, s);
 }
 
 int fa_selftest_bounded_wait(int timeout_us, void* stream) {
