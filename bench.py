@@ -37,8 +37,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from ncu, keyed by the sha256 of the
 # kernel sources they were taken on; a kernel edited since then reports traffic = null.
 NCU_TRAFFIC = {
-    "prefill": {},
-    "decode": {},
+    # profiles/fa_prefill_kernel_mha_causal.md: 543.66 MB read + 48.50 MB written, one launch
+    "prefill": {"24eb617e09b98e34": 592_165_120},
+    # profiles/fa_decode_split_kernel_decode_int8.md: 1107.69 MB read + 3.74 MB written
+    "decode": {"77c2cf5253f1b8fc": 1_111_432_960},
 }
 
 
