@@ -396,10 +396,16 @@ def main():
             },
             "decode": {"value": dec_gbs, "unit": "GB/s", "frac_of_hbm": dec_gbs / world / peaks["hbm_gbs"],
                        "ms_per_call": dec_sum / K},
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
-                         "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+            # The prefill kernel is timed inside a long back-to-back loop of steps under the
+            # power cap, so its denominator is the sustained dense bf16 figure; the burst
+            # figure's fraction is reported beside it.
+            "roofline": {"bound": "tensor", "achieved": achieved,
+                         "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_tflops_sustained"],
+                         "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
                          "traffic": tp, "kernel": "fa_prefill_kernel<128>",
-                         "peak_source": f"{peak_src} bf16 dense (burst)",
+                         "peak_source": f"{peak_src} bf16 dense, sustained (burst "
+                                        f"{peaks['bf16_tflops']:.1f})",
                          "ms_per_launch": pre_avg_s * 1e3},
             "roofline_decode": {"bound": "hbm", "achieved": d_achieved, "peak": peaks["hbm_gbs"],
                                 "unit": "GB/s", "frac": d_achieved / peaks["hbm_gbs"],
