@@ -109,15 +109,22 @@ __device__ __forceinline__ int pow2_exponent_below(float x, int top) {
 
 __device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) << 23); }
 
+#ifndef FA_DECODE_MIN_CTAS
+#define FA_DECODE_MIN_CTAS 3  // CTAs per SM the register allocation must allow
+#endif
+
 template <int D>
-__global__ void __launch_bounds__(128) fa_decode_split_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(128, FA_DECODE_MIN_CTAS) fa_decode_split_kernel(const DecodeParams p) {
   constexpr int KS = D / 16;  // QK k-steps
   constexpr int MT = D / 16;  // PV m-tiles (16 output dims each)
   constexpr int VB = D / 8;   // V bytes per thread per token
-  const int split = blockIdx.x;
-  const int b = blockIdx.y / p.Hkv, kvh = blockIdx.y % p.Hkv;
-  const int head0 = kvh * p.G + blockIdx.z * 8;
-  const int nheads = min(8, p.G - static_cast<int>(blockIdx.z) * 8);
+  // grid (Hkv, splits, B * head blocks): the KV head varies fastest, so CTAs running at the
+  // same time stream the same token rows (all KV heads of a token are contiguous in memory).
+  const int kvh = blockIdx.x, split = blockIdx.y;
+  const int nhb = (p.G + 7) / 8;
+  const int b = static_cast<int>(blockIdx.z) / nhb, hb = static_cast<int>(blockIdx.z) % nhb;
+  const int head0 = kvh * p.G + hb * 8;
+  const int nheads = min(8, p.G - hb * 8);
   const int t_begin = split * p.chunk;
   const int t_end = min(p.Skv, t_begin + p.chunk);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -182,14 +189,15 @@ __global__ void __launch_bounds__(128) fa_decode_split_kernel(const DecodeParams
   const int8_t* vbase = p.v + (static_cast<size_t>(b) * p.Skv * p.Hkv + kvh) * D;
   const int nsteps = (t_end - t_begin + 31) / 32;
 
-  for (int st = warp; st < nsteps; st += 4) {
-    const int T = t_begin + 32 * st;
-    // -- loads (rows past the end are clamped for the address and masked below) --
-    uint32_t kw[2][2][KS];  // [group][row g / g+8][k-step]
-    uint32_t vw[2][4][VB / 4];
-    float ksc[2][2], vsc[2][2];
+  // Each warp takes every 4th 32-token step.  Loads run one step ahead without extra registers:
+  // the next step's K rows are requested as soon as this step's QK^T has consumed the K
+  // registers, the next step's V rows as soon as PV has consumed the V registers.
+  uint32_t kw[2][2][KS];  // [group][row g / g+8][k-step]
+  uint32_t vw[2][4][VB / 4];
+  float ksc[2][2], vsc[2][2];
+  auto load_k = [&](int T) {
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
+    for (int u = 0; u < 2; ++u)
 #pragma unroll
       for (int rr = 0; rr < 2; ++rr) {
         const int tok = min(T + 16 * u + g + 8 * rr, p.Skv - 1);
@@ -207,8 +215,13 @@ __global__ void __launch_bounds__(128) fa_decode_split_kernel(const DecodeParams
           kw[u][rr][7 % KS] = hi.w;
         }
         ksc[u][rr] = ks_row[tok];
-        vsc[u][rr] = vs_row[tok];
       }
+  };
+  auto load_v = [&](int T) {
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) vsc[u][rr] = vs_row[min(T + 16 * u + g + 8 * rr, p.Skv - 1)];
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         const int tok = min(T + 16 * u + 2 * c + (q4 & 1) + 8 * (q4 >> 1), p.Skv - 1);
@@ -226,6 +239,14 @@ __global__ void __launch_bounds__(128) fa_decode_split_kernel(const DecodeParams
         }
       }
     }
+  };
+  if (warp < nsteps) {
+    load_k(t_begin + 32 * warp);
+    load_v(t_begin + 32 * warp);
+  }
+  for (int st = warp; st < nsteps; st += 4) {
+    const int T = t_begin + 32 * st;
+    const bool has_next = st + 4 < nsteps;
 
     // -- S = Kcode . Q^T per 16-token group; x = score in log2 units --
     float x[2][4];
@@ -245,6 +266,7 @@ __global__ void __launch_bounds__(128) fa_decode_split_kernel(const DecodeParams
       x[u][2] = tB < t_end ? sacc[2] * ksc[u][1] * sc0 : -INFINITY;
       x[u][3] = tB < t_end ? sacc[3] * ksc[u][1] * sc1 : -INFINITY;
     }
+    if (has_next) load_k(T + 128);
 
     // -- online softmax per head (columns 2c, 2c+1); max over the warp's 32 tokens --
     float mx0 = fmaxf(fmaxf(x[0][0], x[0][2]), fmaxf(x[1][0], x[1][2]));
@@ -307,6 +329,7 @@ __global__ void __launch_bounds__(128) fa_decode_split_kernel(const DecodeParams
                       pb[u][1]);
       }
     }
+    if (has_next) load_v(T + 128);
   }
 
   // ---- merge the 4 warps ----

@@ -155,9 +155,9 @@ int launch_decode(const void* q, const int8_t* k, const int8_t* v, const float* 
   p.splits = splits;
   p.chunk = (Skv + splits - 1) / splits;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  const long long gy = static_cast<long long>(B) * Hkv;
-  if (gy > 65535 || (p.G + 7) / 8 > 65535 || splits > 0x7fffffff) return FA_ERR_INVALID_ARG;
-  dim3 grid(splits, static_cast<unsigned>(gy), (p.G + 7) / 8);
+  const long long gz = static_cast<long long>(B) * ((p.G + 7) / 8);
+  if (Hkv > 0x7fffffff || splits > 65535 || gz > 65535) return FA_ERR_INVALID_ARG;
+  dim3 grid(Hkv, splits, static_cast<unsigned>(gz));
   fa::fa_decode_split_kernel<D><<<grid, 128, 0, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   fa::CombineParams cp{};
