@@ -37,6 +37,8 @@ def lib():
         L.oracle_attn_brute.argtypes = [_P, _P, _P] + [_I] * 6 + [_D, _I, _I, _P, _P, _P]
         L.oracle_attn_tiled.argtypes = [_P, _P, _P] + [_I] * 6 + [_D, _I, _I, _I, _P, _P]
         L.oracle_decode_int8_rows.argtypes = [_P] * 5 + [_I] * 5 + [_D, _I, _P, _L, _P, _P, _I]
+        L.oracle_decode_int8_paged_rows.argtypes = [_P] * 7 + [_I] * 7 + [_D, _I, _P, _L, _P, _P, _I]
+        L.oracle_decode_int8_paged_rows.restype = _I
         for f in (L.oracle_attn_bf16_rows, L.oracle_attn_f64_rows, L.oracle_attn_brute,
                   L.oracle_attn_tiled, L.oracle_decode_int8_rows):
             f.restype = _I
@@ -148,4 +150,39 @@ def decode_int8(q, kq, vq, ks, vs, scale, num_splits=1, nthreads=0):
     b, h = np.meshgrid(np.arange(B), np.arange(Hq), indexing="ij")
     rows = np.stack([b.ravel(), h.ravel()], axis=1).astype(np.int64)
     o, lse = decode_int8_rows(q, kq, vq, ks, vs, scale, num_splits, rows, nthreads)
+    return o.reshape(B, 1, Hq, D), lse.reshape(B, Hq)
+
+
+def decode_int8_paged_rows(q, kp, vp, ksp, vsp, block_table, seqlens, scale, num_splits, rows,
+                           nthreads=0):
+    """Decode over a paged INT8 KV cache with per-sequence lengths.  q: bf16 bits [B,1,Hq,D];
+    kp/vp: int8 [num_pages,P,Hkv,D]; ksp/vsp: fp32 [num_pages,Hkv,P]; block_table: int32
+    [B,max_pages]; seqlens: int32 [B]; rows: (n, 2) (b, h).  Returns (o [n,D], lse [n])."""
+    B, _, Hq, D = q.shape
+    num_pages, P, Hkv, _ = kp.shape
+    max_pages = block_table.shape[1]
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 2)
+    n = rows.shape[0]
+    o = np.zeros((n, D))
+    lse = np.zeros(n)
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    kp, vp = (np.ascontiguousarray(t, dtype=np.int8) for t in (kp, vp))
+    ksp, vsp = (np.ascontiguousarray(t, dtype=np.float32) for t in (ksp, vsp))
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    sl = np.ascontiguousarray(seqlens, dtype=np.int32)
+    rc = lib().oracle_decode_int8_paged_rows(_ptr(q), _ptr(kp), _ptr(vp), _ptr(ksp), _ptr(vsp),
+                                             _ptr(bt), _ptr(sl), B, Hq, Hkv, P, max_pages,
+                                             num_pages, D, float(scale), int(num_splits),
+                                             _ptr(rows), n, _ptr(o), _ptr(lse), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_decode_int8_paged_rows rejected its arguments")
+    return o, lse
+
+
+def decode_int8_paged(q, kp, vp, ksp, vsp, block_table, seqlens, scale, num_splits=1, nthreads=0):
+    B, _, Hq, D = q.shape
+    b, h = np.meshgrid(np.arange(B), np.arange(Hq), indexing="ij")
+    rows = np.stack([b.ravel(), h.ravel()], axis=1).astype(np.int64)
+    o, lse = decode_int8_paged_rows(q, kp, vp, ksp, vsp, block_table, seqlens, scale, num_splits,
+                                    rows, nthreads)
     return o.reshape(B, 1, Hq, D), lse.reshape(B, Hq)

@@ -32,6 +32,12 @@
 //    dequantised values k_code * k_scale (exact in fp64), one query token per sequence.
 //    With num_splits > 1 it evaluates each key chunk separately and merges the partial
 //    results through their log-sum-exp, the same correction step the online softmax uses.
+//  * Dynamic sequence lengths and a paged KV cache -- "Flash Attention on Ascend: three
+//    techniques", version section (sequences of different lengths in one batch) and "Sparse
+//    attention and MLA operators in ops-transformer", section 2.2 (KV cache pages addressed
+//    through a block_table).  The paged decode
+//    oracle gathers key j of sequence b from page block_table[b][j / P], row j % P, and then
+//    evaluates the same definition over that sequence's own length.
 //
 // Inputs are bf16 bit patterns (widened exactly to fp64), fp64 arrays, or int8 codes with
 // fp32 scales.  Layouts: Q [B, Sq, Hq, D], K/V [B, Skv, Hkv, D], scales [B, Hkv, Skv],
@@ -42,6 +48,7 @@
 #include <cstdint>
 #include <cstring>
 #include <limits>
+#include <utility>
 #include <vector>
 
 namespace {
@@ -348,6 +355,106 @@ int oracle_decode_int8_rows(const uint16_t* q, const int8_t* k, const int8_t* v,
         if (part_l[s] == kNegInf) continue;
         const double w = std::exp(part_l[s] - L);
         for (long t = 0; t < D; ++t) orow[t] += w * part_o[s * D + t];
+      }
+      lse[r] = L;
+    }
+  }
+  return 0;
+}
+
+// Decode over a paged INT8 KV cache with per-sequence lengths.  k/v pages: int8
+// [num_pages, P, Hkv, D]; scales: fp32 [num_pages, Hkv, P]; block_table: int32 [B, max_pages];
+// seqlens: int32 [B].  Key j < seqlens[b] of sequence b is row j % P of page
+// block_table[b][j / P].  rows: (b, h) pairs.  num_splits cuts each sequence into chunks of
+// ceil(seqlens[b] / num_splits) merged by log-sum-exp as in oracle_decode_int8_rows.  A sequence
+// with no key (seqlens[b] == 0) gives O = 0 and LSE = -inf.  Entries of block_table past a
+// sequence's last page are never read.
+int oracle_decode_int8_paged_rows(const uint16_t* q, const int8_t* k, const int8_t* v,
+                                  const float* k_scale, const float* v_scale,
+                                  const int32_t* block_table, const int32_t* seqlens, int B,
+                                  int Hq, int Hkv, int P, int max_pages, int num_pages, int D,
+                                  double scale, int num_splits, const int64_t* rows,
+                                  int64_t nrows, double* o, double* lse, int nthreads) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0 || P <= 0 || max_pages <= 0 ||
+      num_pages <= 0 || D <= 0 || num_splits < 1 || nrows < 0)
+    return -1;
+  if (!q || !k || !v || !k_scale || !v_scale || !block_table || !seqlens) return -1;
+  if (nrows > 0 && (!rows || !o || !lse)) return -1;
+  for (int b = 0; b < B; ++b) {
+    if (seqlens[b] < 0 || seqlens[b] > static_cast<long>(max_pages) * P) return -1;
+    for (long pg = 0; pg < (seqlens[b] + P - 1) / P; ++pg) {
+      const int id = block_table[static_cast<long>(b) * max_pages + pg];
+      if (id < 0 || id >= num_pages) return -1;
+    }
+  }
+  for (int64_t r = 0; r < nrows; ++r)
+    if (rows[2 * r] < 0 || rows[2 * r] >= B || rows[2 * r + 1] < 0 || rows[2 * r + 1] >= Hq)
+      return -1;
+  const long G = Hq / Hkv;
+  if (nthreads <= 0) nthreads = omp_get_max_threads();
+#pragma omp parallel num_threads(nthreads)
+  {
+    std::vector<double> x, part_o(static_cast<size_t>(num_splits) * D), part_l(num_splits);
+#pragma omp for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+      const long b = rows[2 * r], h = rows[2 * r + 1], g = h / G;
+      const long S = seqlens[b];
+      // key j of this sequence: element t of K or V, dequantised
+      auto page_row = [&](long j) {
+        const long pg = block_table[b * max_pages + j / P];
+        return std::make_pair(pg, j % P);
+      };
+      auto kval = [&](long j, long t) {
+        const auto pr = page_row(j);
+        const long idx = ((pr.first * P + pr.second) * Hkv + g) * D + t;
+        return static_cast<double>(k[idx]) *
+               static_cast<double>(k_scale[(pr.first * Hkv + g) * P + pr.second]);
+      };
+      auto vval = [&](long j, long t) {
+        const auto pr = page_row(j);
+        const long idx = ((pr.first * P + pr.second) * Hkv + g) * D + t;
+        return static_cast<double>(v[idx]) *
+               static_cast<double>(v_scale[(pr.first * Hkv + g) * P + pr.second]);
+      };
+      const long chunk = (S + num_splits - 1) / num_splits;
+      x.assign(S, kNegInf);
+      for (int s = 0; s < num_splits; ++s) {
+        const long j0 = std::min<long>(S, s * chunk), j1 = std::min<long>(S, (s + 1) * chunk);
+        double* po = part_o.data() + static_cast<size_t>(s) * D;
+        for (long t = 0; t < D; ++t) po[t] = 0.0;
+        if (j0 >= j1) {
+          part_l[s] = kNegInf;
+          continue;
+        }
+        // the definition over keys [j0, j1): scores, their max, exp-sum, weighted V sum
+        double m = kNegInf;
+        for (long j = j0; j < j1; ++j) {
+          double dot = 0.0;
+          for (long t = 0; t < D; ++t) dot += widen_bf16(q[(b * Hq + h) * D + t]) * kval(j, t);
+          x[j] = scale * dot;
+          m = std::max(m, x[j]);
+        }
+        double l = 0.0;
+        for (long j = j0; j < j1; ++j) {
+          const double pj = std::exp(x[j] - m);
+          l += pj;
+          for (long t = 0; t < D; ++t) po[t] += pj * vval(j, t);
+        }
+        for (long t = 0; t < D; ++t) po[t] /= l;
+        part_l[s] = m + std::log(l);
+      }
+      double mx = kNegInf;
+      for (int s = 0; s < num_splits; ++s) mx = std::max(mx, part_l[s]);
+      double sum = 0.0;
+      for (int s = 0; s < num_splits; ++s)
+        if (part_l[s] != kNegInf) sum += std::exp(part_l[s] - mx);
+      const double L = mx + std::log(sum);
+      double* orow = o + r * D;
+      for (long t = 0; t < D; ++t) orow[t] = 0.0;
+      for (int s = 0; s < num_splits; ++s) {
+        if (part_l[s] == kNegInf) continue;
+        const double w = std::exp(part_l[s] - L);
+        for (long t = 0; t < D; ++t) orow[t] += w * part_o[static_cast<size_t>(s) * D + t];
       }
       lse[r] = L;
     }

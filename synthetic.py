@@ -18,7 +18,16 @@ This module holds no attention arithmetic. It only draws numbers and names workl
   Llama-2-7B 32/32, Mistral-7B 32/8, Falcon-180B 232/1) plus a tiny parity case and
   an INT8-KV decode case.
 
-Seeds are ``20260 + 10 * workload_index + tensor_index`` with Q=0, K=1, V=2.
+* ``PAGED_WORKLOADS`` / ``make_paged_decode_inputs`` -- decode over a paged INT8 cache with a
+  mix of sequence lengths in one batch ("Flash Attention on Ascend: three techniques", version
+  section: sequences of different lengths computed together; "Sparse attention and MLA operators
+  in ops-transformer", section 2.2: KV pages addressed through a block_table).  Lengths are uniform integers in
+  [min_len, max_len] (splitmix64 value modulo the range; the modulo bias is below 2^-40), and
+  the physical pages are handed out in the order of a seeded random permutation, so that each
+  sequence's pages are scattered over the pool as in a long-running cache.
+
+Seeds are ``20260 + 10 * workload_index + tensor_index`` with Q=0, K=1, V=2 (paged workloads
+add lengths=3 and page permutation=4).
 """
 from __future__ import annotations
 
@@ -247,3 +256,84 @@ def sample_rows(B: int, H: int, S: int, seed: int, n_random: int, window: int = 
         fixed.add((int(r[0] % np.uint64(B)), int(r[1] % np.uint64(H)), int(r[2] % np.uint64(S))))
     rows = np.array(sorted(fixed), dtype=np.int64)
     return rows
+
+
+# ---------------------------------------------------------------------------------------
+# Paged KV cache with per-sequence lengths.
+# Layouts: K/V pages int8 [num_pages, P, Hkv, D]; scales fp32 [num_pages, Hkv, P];
+# block_table int32 [B, max_pages] (entries past a sequence's last page are -1 and unused);
+# seqlens int32 [B].
+# ---------------------------------------------------------------------------------------
+@dataclass(frozen=True)
+class PagedDecodeWorkload:
+    name: str
+    index: int
+    B: int
+    Hq: int
+    Hkv: int
+    D: int
+    page_size: int
+    min_len: int
+    max_len: int
+    num_splits: int = 16
+    note: str = ""
+
+    @property
+    def scale(self) -> float:
+        return float(np.float32(1.0 / math.sqrt(self.D)))
+
+    @property
+    def max_pages(self) -> int:
+        return -(-self.max_len // self.page_size)
+
+    def seed(self, tensor_index: int) -> int:
+        return 20260 + 10 * self.index + tensor_index
+
+
+PAGED_WORKLOADS = {
+    "decode_int8_paged": PagedDecodeWorkload(
+        "decode_int8_paged", 6, 16, 32, 8, 128, 64, 1, 32768, 16,
+        note="GQA decode over a paged INT8 cache, lengths uniform in [1, 32768]"),
+}
+
+
+def paged_layout(w: PagedDecodeWorkload, seqlens=None):
+    """(seqlens int32 [B], block_table int32 [B, max_pages], num_pages).  ``seqlens`` may be
+    given explicitly; otherwise it is drawn uniformly from [min_len, max_len]."""
+    if seqlens is None:
+        u = splitmix64(w.seed(3), 0, w.B)
+        span = np.uint64(w.max_len - w.min_len + 1)
+        seqlens = (np.uint64(w.min_len) + u % span).astype(np.int64)
+    seqlens = np.asarray(seqlens, dtype=np.int64)
+    assert seqlens.shape == (w.B,) and seqlens.min() >= 0 and seqlens.max() <= w.max_len
+    npages = -(-seqlens // w.page_size)
+    num_pages = max(1, int(npages.sum()))
+    perm = np.argsort(splitmix64(w.seed(4), 0, num_pages), kind="stable").astype(np.int32)
+    bt = np.full((w.B, w.max_pages), -1, dtype=np.int32)
+    off = 0
+    for b in range(w.B):
+        bt[b, : npages[b]] = perm[off: off + npages[b]]
+        off += int(npages[b])
+    return seqlens.astype(np.int32), bt, num_pages
+
+
+def make_paged_decode_inputs(w: PagedDecodeWorkload, seqlens=None):
+    """q bf16 bits [B,1,Hq,D]; K/V int8 pages, fp32 scale pages, block_table, seqlens."""
+    sl, bt, num_pages = paged_layout(w, seqlens)
+    q = normal_bf16(w.seed(0), (w.B, 1, w.Hq, w.D))
+    shape = (num_pages, w.page_size, w.Hkv, w.D)
+    kp, ksp = quantize_int8_per_token(normal_bf16(w.seed(1), shape))
+    vp, vsp = quantize_int8_per_token(normal_bf16(w.seed(2), shape))
+    return q, kp, vp, ksp, vsp, bt, sl
+
+
+def make_paged_decode_inputs_torch(w: PagedDecodeWorkload, device, seqlens=None):
+    """The same inputs drawn with the torch generator on ``device`` (large workloads)."""
+    import torch
+    sl, bt, num_pages = paged_layout(w, seqlens)
+    q = normal_bf16_torch(w.seed(0), (w.B, 1, w.Hq, w.D), device)
+    shape = (num_pages, w.page_size, w.Hkv, w.D)
+    kp, ksp = quantize_int8_per_token_torch(normal_bf16_torch(w.seed(1), shape, device))
+    vp, vsp = quantize_int8_per_token_torch(normal_bf16_torch(w.seed(2), shape, device))
+    return (q, kp, vp, ksp, vsp, torch.from_numpy(bt).to(device),
+            torch.from_numpy(sl).to(device))
