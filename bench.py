@@ -6,6 +6,8 @@ One step = one pass of the whole path over one batch of synthetic input:
     headline metric is quoted on (attention forward TFLOP/s);
   * decode   (fa_decode_int8, split kernel + combine kernel): B=16, Hq=32, Hkv=8, Skv=32768,
     D=128, INT8 KV cache with per-token scales, 16 splits (KV-read GB/s).
+After the timed steps, a short loop of its own times the paged, variable-length decode
+(fa_decode_int8_paged) and reports it under "paged_decode"; it is not part of the step.
 Inputs are seeded synthetic N(0,1) draws (see synthetic.py) resident in HBM; both inputs are
 larger than the 126 MB L2 (prefill 268 MB, decode 1.1 GB), so no flush is needed between steps.
 
@@ -79,6 +81,45 @@ def decode_bytes(w) -> int:
     scales = 2 * w.B * w.Hkv * w.Skv * 4
     qo = 2 * w.B * w.Hq * w.D * 2
     return kv + scales + qo + w.B * w.Hq * 4
+
+
+def paged_decode_bytes(w, seqlens) -> int:
+    """Algorithmic bytes of one paged decode call: the int8 K and V rows and fp32 scales of every
+    cached key, the block-table entries of the pages in use, the lengths, q in, o out, LSE."""
+    import numpy as np
+    sl = np.asarray(seqlens, dtype=np.int64)
+    keys = int(sl.sum())
+    pages = int((-(-sl // w.page_size)).sum())
+    kv = 2 * keys * w.Hkv * w.D + 2 * keys * w.Hkv * 4
+    return kv + 4 * pages + 4 * w.B + 2 * w.B * w.Hq * w.D * 2 + w.B * w.Hq * 4
+
+
+def measure_paged_decode(fa, synthetic, torch, dev, stream, steps: int, warmup: int):
+    """Time fa_decode_int8_paged on the paged workload (its own short loop after the step loop).
+    Returns (ms per call averaged over ``steps`` launches, algorithmic bytes per call)."""
+    w = synthetic.PAGED_WORKLOADS["decode_int8_paged"]
+    q, kp, vp, ksp, vsp, bt, sl = synthetic.make_paged_decode_inputs_torch(w, dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(fa.fa_decode_int8_workspace_bytes(w.B, w.Hq, w.D, w.num_splits),
+                     dtype=torch.uint8, device=dev)
+
+    def call():
+        fa.fa_decode_int8_paged(q, kp, vp, ksp, vsp, bt, sl, num_splits=w.num_splits,
+                                scale=w.scale, o=o, lse=lse, workspace=ws, stream=stream)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        call()
+    b.record(stream)
+    torch.cuda.synchronize()
+    if fa.fa_device_status() != 0:
+        raise RuntimeError("the paged decode reported a device-side error")
+    return a.elapsed_time(b) / steps, paged_decode_bytes(w, sl.cpu().numpy())
 
 
 class ClockSampler:
@@ -329,6 +370,11 @@ def main():
     achieved = flops / pre_avg_s / 1e12
     d_achieved = dbytes / dec_avg_s / 1e9
 
+    # ---- the paged, variable-length decode (a further row of the path), its own short loop ----
+    pg_ms, pg_bytes = measure_paged_decode(fa, synthetic, torch, dev, stream,
+                                           steps=min(K, 200), warmup=max(3, args.warmup // 4))
+    pg_ms = max_over_ranks(pg_ms)
+
     # ---- end to end through the public API, host buffers, copies inside the timed region ----
     e2e = None
     if args.e2e_steps > 0:
@@ -413,6 +459,15 @@ def main():
                                 "kernel": "fa_decode_split_kernel<128> + fa_decode_combine_kernel<128>",
                                 "peak_source": f"{peak_src} copy bandwidth",
                                 "ms_per_call": dec_avg_s * 1e3},
+            "paged_decode": {
+                "workload": "decode_int8_paged: B=16, Hq=32, Hkv=8, D=128, INT8 KV in 64-token "
+                            "pages scattered over the pool, lengths uniform in [1, 32768] "
+                            f"({pg_bytes / 1e6:.1f} MB per call), 16 splits",
+                "kernel": "fa_decode_split_kernel<128, paged> + fa_decode_combine_kernel<128>",
+                "ms_per_call": pg_ms, "achieved": pg_bytes / (pg_ms * 1e-3) / 1e9,
+                "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                "frac": pg_bytes / (pg_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "launches": 2 * min(K, 200)},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 3 * K,

@@ -19,7 +19,10 @@
  *   - causal and sliding-window masks (each query sees its W nearest keys, itself included):
  *     same page, sliding-window section;
  *   - decode over an INT8 KV cache computed without decompressing it first: "Flash
- *     Attention on Ascend: three techniques", section 3 (KV compression).
+ *     Attention on Ascend: three techniques", section 3 (KV compression);
+ *   - a paged KV cache addressed through a block_table, with one length per sequence:
+ *     "Sparse attention and MLA operators in ops-transformer", section 2.2, and the
+ *     three-techniques page, version section (dynamic sequence length).
  *
  * Conventions shared by every entry point
  *   - All tensor arguments are DEVICE pointers owned by the caller, contiguous, 16-byte
@@ -29,7 +32,8 @@
  *   - Calls validate their arguments synchronously and enqueue their kernels asynchronously on
  *     `stream` (a cudaStream_t; NULL is the legacy default stream).  Errors that happen on the
  *     device surface at the caller's next synchronisation; fa_device_status() reports the
- *     library's own device-side failures (a bounded wait that gave up).
+ *     library's own device-side failures (a bounded wait that gave up, an out-of-range index
+ *     read from device memory).
  *   - Thread safety: calls may be made from several host threads; they share no mutable
  *     state beyond one-time initialisation, which is guarded.
  */
@@ -56,7 +60,9 @@ typedef enum {
   FA_ERR_ALIGNMENT = -3,   /* a tensor pointer is not 16-byte aligned */
   FA_ERR_WORKSPACE = -4,   /* decode workspace missing or smaller than required */
   FA_ERR_CUDA = -5,        /* a CUDA runtime/driver call or a kernel launch failed */
-  FA_ERR_TIMEOUT = -6      /* a kernel gave up a bounded wait (reported by fa_device_status) */
+  FA_ERR_TIMEOUT = -6,     /* a kernel gave up a bounded wait (reported by fa_device_status) */
+  FA_ERR_DEVICE_INDEX = -7 /* a page id or sequence length read on the device was out of range
+                              (reported by fa_device_status) */
 } fa_status;
 
 /*
@@ -137,14 +143,53 @@ FA_API int fa_decode_int8_noalloc(const void* q, const int8_t* k, const int8_t* 
                                   int B, int Hq, int Hkv, int Skv, int D, float scale,
                                   int num_splits, void* stream);
 
+/*
+ * Decode step over a PAGED INT8 KV cache with one length per sequence.
+ * Sources: the KV cache stored in pages that a block_table maps to each sequence ("Sparse
+ * attention and MLA operators in ops-transformer", section 2.2, paged attention through a
+ * block_table); sequences of different lengths computed in one batch ("Flash Attention on
+ * Ascend: three techniques", version section, dynamic sequence length); the INT8 cache used
+ * without decompressing it first (same page, section 3).
+ *   q        bf16 [B, 1, Hq, D]
+ *   k_pages, v_pages  int8 [num_pages, page_size, Hkv, D]   a pool of pages of page_size tokens
+ *   k_scale_pages, v_scale_pages  fp32 [num_pages, Hkv, page_size]  one scale per (token, head)
+ *   block_table  int32 [B, max_pages_per_seq] (device): key j of sequence b is row
+ *            j % page_size of page block_table[b][j / page_size].  Entries past a sequence's
+ *            last page are never read and may hold anything.
+ *   seqlens  int32 [B] (device): number of keys of each sequence, 0 .. max_pages_per_seq *
+ *            page_size.  A sequence with 0 keys gets O = 0 and LSE = -inf.
+ *   o, lse   as for fa_decode_int8.
+ *   page_size  a power of two, 16 .. 65536; max_pages_per_seq * page_size <= 2^30.
+ *   num_pages  number of pages in the pool (page ids are 0 .. num_pages - 1).
+ *   num_splits >= 1: each sequence's keys are cut into num_splits chunks of
+ *            ceil(seqlens[b] / num_splits) keys rounded up to a multiple of 16; chunks are
+ *            merged through their log-sum-exp as in fa_decode_int8.
+ *   workspace  at least fa_decode_int8_workspace_bytes(B, Hq, D, num_splits) bytes.
+ * block_table and seqlens need 4-byte alignment; every other tensor 16-byte alignment.
+ * The lengths and page ids live in device memory, so they are checked on the device: an id
+ * outside 0 .. num_pages - 1 or a length outside the range above is replaced by a valid one (no
+ * access ever leaves the pool) and recorded, and the next fa_device_status() returns
+ * FA_ERR_DEVICE_INDEX; the outputs of that call are then undefined.
+ * D must be 64 or 128; Hq must be a multiple of Hkv.  Returns FA_OK or an fa_status error code;
+ * nothing is launched on error.
+ */
+FA_API int fa_decode_int8_paged(const void* q, const int8_t* k_pages, const int8_t* v_pages,
+                                const float* k_scale_pages, const float* v_scale_pages,
+                                const int32_t* block_table, const int32_t* seqlens, void* o,
+                                float* lse, int B, int Hq, int Hkv, int page_size,
+                                int max_pages_per_seq, int num_pages, int D, float scale,
+                                int num_splits, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
 /* Static, human-readable name of a status code.  Never NULL. */
 FA_API const char* fa_status_string(int status);
 
 /*
  * Synchronises `stream`, then reads and clears the library's device status word on the current
  * device.  Returns FA_ERR_TIMEOUT if a kernel launched by this library gave up a bounded wait
- * since the last call (its outputs are then undefined), FA_ERR_CUDA if the synchronisation
- * failed, else FA_OK.
+ * since the last call, else FA_ERR_DEVICE_INDEX if a kernel met an out-of-range page id or
+ * sequence length (the outputs of such a call are undefined), FA_ERR_CUDA if the
+ * synchronisation failed, else FA_OK.
  */
 FA_API int fa_device_status(void* stream);
 

@@ -31,7 +31,8 @@ def declared_functions():
 def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("fa_fwd", "fa_decode_int8", "fa_decode_int8_workspace_bytes", "fa_status_string",
-              "fa_device_status", "fa_selftest_bounded_wait"):
+              "fa_device_status", "fa_selftest_bounded_wait", "fa_decode_int8_noalloc",
+              "fa_decode_int8_paged"):
         assert n in names
 
 
@@ -101,6 +102,37 @@ def dec(L, q=FAKE, k=FAKE, v=FAKE, ks=FAKE, vs=FAKE, o=FAKE, lse=None, B=2, Hq=8
 ])
 def test_decode_rejects(L, kw, code):
     assert dec(L, **kw) == code
+
+
+def paged(L, q=FAKE, k=FAKE, v=FAKE, ks=FAKE, vs=FAKE, bt=FAKE, sl=FAKE, o=FAKE, lse=None, B=2,
+          Hq=8, Hkv=2, P=64, max_pages=8, num_pages=16, D=128, scale=0.1, splits=4, ws=FAKE,
+          ws_bytes=None):
+    if ws_bytes is None:
+        ws_bytes = L.fa_decode_int8_workspace_bytes(B, Hq, D, splits)
+    return L.fa_decode_int8_paged(q, k, v, ks, vs, bt, sl, o, lse, B, Hq, Hkv, P, max_pages,
+                                  num_pages, D, scale, splits, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(bt=None), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(sl=None), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(P=48), fa.STATUS["FA_ERR_INVALID_ARG"]),        # not a power of two
+    (dict(P=8), fa.STATUS["FA_ERR_INVALID_ARG"]),         # below 16
+    (dict(P=1 << 17), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(max_pages=0), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(num_pages=0), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(max_pages=1 << 25, P=64), fa.STATUS["FA_ERR_INVALID_ARG"]),  # > 2^30 keys
+    (dict(Hq=6, Hkv=4), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(splits=0), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(D=96), fa.STATUS["FA_ERR_UNSUPPORTED"]),
+    (dict(k=FAKE + 8), fa.STATUS["FA_ERR_ALIGNMENT"]),
+    (dict(bt=FAKE + 2), fa.STATUS["FA_ERR_ALIGNMENT"]),
+    (dict(sl=FAKE + 1), fa.STATUS["FA_ERR_ALIGNMENT"]),
+    (dict(ws=None), fa.STATUS["FA_ERR_WORKSPACE"]),
+    (dict(ws_bytes=64), fa.STATUS["FA_ERR_WORKSPACE"]),
+])
+def test_paged_decode_rejects(L, kw, code):
+    assert paged(L, **kw) == code
 
 
 def test_workspace_bytes(L):

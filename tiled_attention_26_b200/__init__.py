@@ -12,9 +12,9 @@ import ctypes
 import math
 import os
 
-__all__ = ["FaError", "lib", "fa_fwd", "fa_decode_int8", "fa_decode_int8_workspace_bytes",
-           "fa_status_string", "fa_device_status", "fa_selftest_bounded_wait", "LIB_PATH",
-           "STATUS"]
+__all__ = ["FaError", "lib", "fa_fwd", "fa_decode_int8", "fa_decode_int8_paged",
+           "fa_decode_int8_workspace_bytes", "fa_status_string", "fa_device_status",
+           "fa_selftest_bounded_wait", "LIB_PATH", "STATUS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
 
@@ -26,6 +26,7 @@ STATUS = {
     "FA_ERR_WORKSPACE": -4,
     "FA_ERR_CUDA": -5,
     "FA_ERR_TIMEOUT": -6,
+    "FA_ERR_DEVICE_INDEX": -7,
 }
 
 
@@ -56,6 +57,8 @@ def lib() -> ctypes.CDLL:
         L.fa_decode_int8_workspace_bytes.restype = _Z
         L.fa_decode_int8.argtypes = [_P] * 7 + [_I] * 5 + [_F, _I, _P, _Z, _P]
         L.fa_decode_int8.restype = _I
+        L.fa_decode_int8_paged.argtypes = [_P] * 9 + [_I] * 7 + [_F, _I, _P, _Z, _P]
+        L.fa_decode_int8_paged.restype = _I
         L.fa_status_string.argtypes = [_I]
         L.fa_status_string.restype = ctypes.c_char_p
         L.fa_device_status.argtypes = [_P]
@@ -162,6 +165,52 @@ def fa_decode_int8(q, k, v, k_scale, v_scale, num_splits: int = 16, scale: float
                               workspace.numel() * workspace.element_size(), _stream_ptr(stream))
     if rc != 0:
         raise FaError(rc, "fa_decode_int8")
+    return o, lse
+
+
+def fa_decode_int8_paged(q, k_pages, v_pages, k_scale_pages, v_scale_pages, block_table,
+                         seqlens, num_splits: int = 16, scale: float | None = None, o=None,
+                         lse=None, workspace=None, return_lse: bool = True, stream=None):
+    """Decode step over a paged INT8 KV cache with one length per sequence.
+    q: bf16 [B, 1, Hq, D]; k_pages, v_pages: int8 [num_pages, P, Hkv, D]; k_scale_pages,
+    v_scale_pages: fp32 [num_pages, Hkv, P]; block_table: int32 [B, max_pages]; seqlens: int32
+    [B] (both on the device).  Returns ``(o, lse)`` with o bf16 [B, 1, Hq, D], lse fp32 [B, Hq]."""
+    import torch
+    B, one, Hq, D = q.shape
+    if one != 1:
+        raise ValueError("decode takes one query token per sequence")
+    if k_pages.dim() != 4 or block_table.dim() != 2:
+        raise ValueError("k_pages must be [num_pages, P, Hkv, D], block_table [B, max_pages]")
+    num_pages, P, Hkv = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    max_pages = block_table.shape[1]
+    dev = q.device
+    _check(q, "q", torch.bfloat16, (B, 1, Hq, D), dev)
+    _check(k_pages, "k_pages", torch.int8, (num_pages, P, Hkv, D), dev)
+    _check(v_pages, "v_pages", torch.int8, (num_pages, P, Hkv, D), dev)
+    _check(k_scale_pages, "k_scale_pages", torch.float32, (num_pages, Hkv, P), dev)
+    _check(v_scale_pages, "v_scale_pages", torch.float32, (num_pages, Hkv, P), dev)
+    _check(block_table, "block_table", torch.int32, (B, max_pages), dev)
+    _check(seqlens, "seqlens", torch.int32, (B,), dev)
+    if o is None:
+        o = torch.empty_like(q)
+    _check(o, "o", torch.bfloat16, (B, 1, Hq, D), dev)
+    if lse is None and return_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    if lse is not None:
+        _check(lse, "lse", torch.float32, (B, Hq), dev)
+    need = fa_decode_int8_workspace_bytes(B, Hq, D, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    rc = lib().fa_decode_int8_paged(
+        q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), k_scale_pages.data_ptr(),
+        v_scale_pages.data_ptr(), block_table.data_ptr(), seqlens.data_ptr(), o.data_ptr(),
+        lse.data_ptr() if lse is not None else None, B, Hq, Hkv, P, max_pages, num_pages, D,
+        float(scale), int(num_splits), workspace.data_ptr(),
+        workspace.numel() * workspace.element_size(), _stream_ptr(stream))
+    if rc != 0:
+        raise FaError(rc, "fa_decode_int8_paged")
     return o, lse
 
 

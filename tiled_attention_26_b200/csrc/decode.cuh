@@ -22,6 +22,16 @@
 // runs on the accumulator fragments.  The 4 warps merge through shared memory and the CTA
 // writes a normalised partial output and its log-sum-exp to the workspace.
 //
+// Paged variant (kPaged): the cache is a pool of pages of P tokens (P a power of two >= 16),
+// [num_pages, P, Hkv, D] codes and [num_pages, Hkv, P] scales, and sequence b owns the pages
+// listed in block_table[b] ("Sparse attention and MLA operators in ops-transformer", section 2.2:
+// the KV cache addressed through a block_table) and has its own length seqlens[b], read on the
+// device ("Flash Attention on Ascend: three techniques", version section: sequences of different
+// lengths in one batch).  Each split covers ceil(len / splits) keys rounded up to 16, so every
+// 16-token group of a step lies inside one page: the page is looked up once per group.  Page ids
+// and lengths are range-checked; a bad one is recorded in the device status word and replaced by
+// a valid one, so a corrupt table never makes the kernel read outside the pool.
+//
 // Merge step (fa_decode_combine_kernel): L = log sum_s exp(L_s), O = sum_s exp(L_s - L) O_s.
 #pragma once
 
@@ -31,14 +41,18 @@ namespace fa {
 
 struct DecodeParams {
   const uint16_t* q;  // bf16 [B, 1, Hq, D]
-  const int8_t* k;    // [B, Skv, Hkv, D]
+  const int8_t* k;    // [B, Skv, Hkv, D]; paged: [num_pages, P, Hkv, D]
   const int8_t* v;
-  const float* k_scale;  // [B, Hkv, Skv]
+  const float* k_scale;  // [B, Hkv, Skv]; paged: [num_pages, Hkv, P]
   const float* v_scale;
   float* o_part;    // [splits, B, Hq, D]
   float* lse_part;  // [splits, B, Hq]
   int B, Hq, Hkv, Skv, G, splits, chunk;
   float scale_log2;
+  // paged cache only
+  const int32_t* block_table;  // [B, max_pages]
+  const int32_t* seqlens;      // [B]
+  int max_pages, num_pages, page_shift;  // P = 1 << page_shift
 };
 
 struct CombineParams {
@@ -109,24 +123,50 @@ __device__ __forceinline__ int pow2_exponent_below(float x, int top) {
 
 __device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) << 23); }
 
+#ifndef FA_PAGED_SMEM_PAGES
+#define FA_PAGED_SMEM_PAGES 1  // stage each split's page ids in shared memory
+#endif
+
+#ifndef FA_PAGED_VMAX_BATCH
+#define FA_PAGED_VMAX_BATCH 1
+#endif
+
+#ifndef FA_DECODE_PDL
+#define FA_DECODE_PDL 1  // launch the merge kernel as a programmatic dependent of the split kernel
+#endif
+
 #ifndef FA_DECODE_MIN_CTAS
 #define FA_DECODE_MIN_CTAS 3  // CTAs per SM the register allocation must allow
 #endif
 
-template <int D>
+template <int D, bool kPaged>
 __global__ void __launch_bounds__(128, FA_DECODE_MIN_CTAS) fa_decode_split_kernel(const DecodeParams p) {
   constexpr int KS = D / 16;  // QK k-steps
   constexpr int MT = D / 16;  // PV m-tiles (16 output dims each)
   constexpr int VB = D / 8;   // V bytes per thread per token
   // grid (Hkv, splits, B * head blocks): the KV head varies fastest, so CTAs running at the
   // same time stream the same token rows (all KV heads of a token are contiguous in memory).
+  // the merge kernel may be scheduled as soon as every CTA of this grid has started
+  asm volatile("griddepcontrol.launch_dependents;");
   const int kvh = blockIdx.x, split = blockIdx.y;
   const int nhb = (p.G + 7) / 8;
   const int b = static_cast<int>(blockIdx.z) / nhb, hb = static_cast<int>(blockIdx.z) % nhb;
   const int head0 = kvh * p.G + hb * 8;
   const int nheads = min(8, p.G - hb * 8);
-  const int t_begin = split * p.chunk;
-  const int t_end = min(p.Skv, t_begin + p.chunk);
+  int len = p.Skv, chunk = p.chunk;
+  const int32_t* bt_row = nullptr;
+  if constexpr (kPaged) {
+    const int cap = p.max_pages << p.page_shift;
+    len = p.seqlens[b];
+    if (len < 0 || len > cap) {
+      if (threadIdx.x == 0) atomicOr(&g_fa_device_status, kDevStatusBadIndex);
+      len = max(0, min(len, cap));
+    }
+    chunk = ((len + p.splits - 1) / p.splits + 15) & ~15;
+    bt_row = p.block_table + static_cast<size_t>(b) * p.max_pages;
+  }
+  const int t_begin = split * chunk;
+  const int t_end = min(len, t_begin + chunk);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
 
@@ -134,12 +174,86 @@ __global__ void __launch_bounds__(128, FA_DECODE_MIN_CTAS) fa_decode_split_kerne
   __shared__ float sm_m[4][8], sm_l[4][8];
   __shared__ float sm_o[4][8][D];
 
+  const size_t row_stride = static_cast<size_t>(p.Hkv) * D;  // bytes between tokens
+  const int pmask = (1 << p.page_shift) - 1;
+  // physical page of key t (t < len): checked against the pool, never outside it
+  auto checked_page = [&](int slot) -> int {
+    int pg = bt_row[slot];
+    if (static_cast<unsigned>(pg) >= static_cast<unsigned>(p.num_pages)) {
+      atomicOr(&g_fa_device_status, kDevStatusBadIndex);
+      pg = 0;
+    }
+    return pg;
+  };
+#if FA_PAGED_SMEM_PAGES
+  // The split's page ids are staged in shared memory once (checked there), so the loads of a
+  // step never wait on a dependent global load.  A split spanning more pages than the stage
+  // holds reads the table directly.
+  constexpr int kPageStage = 512;
+  __shared__ int sm_pages[kPageStage];
+  const int first_slot = kPaged ? (t_begin >> p.page_shift) : 0;
+  const int n_slots = (kPaged && t_end > t_begin) ? ((t_end - 1) >> p.page_shift) - first_slot + 1 : 0;
+  const bool staged = n_slots <= kPageStage;
+  if constexpr (kPaged) {
+    if (staged)
+      for (int i = threadIdx.x; i < n_slots; i += 128) sm_pages[i] = checked_page(first_slot + i);
+    __syncthreads();
+  }
+  auto page_of = [&](int t) -> int {
+    const int slot = t >> p.page_shift;
+    return staged ? sm_pages[slot - first_slot] : checked_page(slot);
+  };
+#else
+  auto page_of = [&](int t) -> int { return checked_page(t >> p.page_shift); };
+#endif
+  // offset of (page pg, kv head kvh, row r) in the [num_pages, Hkv, P] scale arrays
+  auto page_scale_index = [&](int pg, int r) -> size_t {
+    return ((static_cast<size_t>(pg) * p.Hkv + kvh) << p.page_shift) + r;
+  };
+  // paged: code row and scale pointers of the 16-token group that starts at key gs0.  A group
+  // past the split's last key is replaced by the split's last group (its extra keys are masked),
+  // so every page looked up belongs to this split.
+  const int last16 = (t_end - 1) & ~15;
+  auto group_base = [&](int gs0, const int8_t* codes, const float* scales, const int8_t*& rows,
+                        const float*& sc) {
+    const int gs = min(gs0, last16);
+    const int pg = page_of(gs);
+    const int r0 = gs & pmask;
+    rows = codes + ((static_cast<size_t>(pg) << p.page_shift) + r0) * row_stride +
+           static_cast<size_t>(kvh) * D;
+    sc = scales + page_scale_index(pg, r0);
+  };
+
   const float* ks_row = p.k_scale + (static_cast<size_t>(b) * p.Hkv + kvh) * p.Skv;
   const float* vs_row = p.v_scale + (static_cast<size_t>(b) * p.Hkv + kvh) * p.Skv;
 
   // ---- P' = p * v_scale * 2^E stays below 2^15 in fp16: E from the split's largest v_scale ----
   float vmax = 0.f;
-  for (int t = t_begin + threadIdx.x; t < t_end; t += 128) vmax = fmaxf(vmax, vs_row[t]);
+  if constexpr (kPaged) {
+#if FA_PAGED_VMAX_BATCH
+    // 8 keys per thread per round: all page ids, then all scales, so each round waits for two
+    // memory latencies instead of sixteen
+    for (int t0 = t_begin + threadIdx.x; t0 < t_end; t0 += 128 * 8) {
+      int pg[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int t = min(t0 + 128 * i, t_end - 1);
+        pg[i] = page_of(t);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int t = t0 + 128 * i;
+        const float sv = p.v_scale[page_scale_index(pg[i], min(t, t_end - 1) & pmask)];
+        vmax = fmaxf(vmax, sv);
+      }
+    }
+#else
+    for (int t = t_begin + threadIdx.x; t < t_end; t += 128)
+      vmax = fmaxf(vmax, p.v_scale[page_scale_index(page_of(t), t & pmask)]);
+#endif
+  } else {
+    for (int t = t_begin + threadIdx.x; t < t_end; t += 128) vmax = fmaxf(vmax, vs_row[t]);
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
   if (lane == 0) sm_red[warp] = vmax;
@@ -184,7 +298,6 @@ __global__ void __launch_bounds__(128, FA_DECODE_MIN_CTAS) fa_decode_split_kerne
   for (int mt = 0; mt < MT; ++mt) oacc[mt][0] = oacc[mt][1] = oacc[mt][2] = oacc[mt][3] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
-  const size_t row_stride = static_cast<size_t>(p.Hkv) * D;  // bytes between tokens
   const int8_t* kbase = p.k + (static_cast<size_t>(b) * p.Skv * p.Hkv + kvh) * D;
   const int8_t* vbase = p.v + (static_cast<size_t>(b) * p.Skv * p.Hkv + kvh) * D;
   const int nsteps = (t_end - t_begin + 31) / 32;
@@ -197,11 +310,15 @@ __global__ void __launch_bounds__(128, FA_DECODE_MIN_CTAS) fa_decode_split_kerne
   float ksc[2][2], vsc[2][2];
   auto load_k = [&](int T) {
 #pragma unroll
-    for (int u = 0; u < 2; ++u)
+    for (int u = 0; u < 2; ++u) {
+      const int8_t* gk = nullptr;
+      const float* gks = nullptr;
+      if constexpr (kPaged) group_base(T + 16 * u, p.k, p.k_scale, gk, gks);
 #pragma unroll
       for (int rr = 0; rr < 2; ++rr) {
-        const int tok = min(T + 16 * u + g + 8 * rr, p.Skv - 1);
-        const int8_t* row = kbase + static_cast<size_t>(tok) * row_stride;
+        const int tok = min(T + 16 * u + g + 8 * rr, len - 1);
+        const int8_t* row = kPaged ? gk + static_cast<size_t>(g + 8 * rr) * row_stride
+                                   : kbase + static_cast<size_t>(tok) * row_stride;
         const uint4 lo = ldg_stream16(row + 16 * c);
         kw[u][rr][0] = lo.x;
         kw[u][rr][1] = lo.y;
@@ -214,18 +331,26 @@ __global__ void __launch_bounds__(128, FA_DECODE_MIN_CTAS) fa_decode_split_kerne
           kw[u][rr][6 % KS] = hi.z;
           kw[u][rr][7 % KS] = hi.w;
         }
-        ksc[u][rr] = ks_row[tok];
+        ksc[u][rr] = kPaged ? gks[g + 8 * rr] : ks_row[tok];
       }
+    }
   };
   auto load_v = [&](int T) {
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
+      const int8_t* gv = nullptr;
+      const float* gvs = nullptr;
+      if constexpr (kPaged) group_base(T + 16 * u, p.v, p.v_scale, gv, gvs);
 #pragma unroll
-      for (int rr = 0; rr < 2; ++rr) vsc[u][rr] = vs_row[min(T + 16 * u + g + 8 * rr, p.Skv - 1)];
+      for (int rr = 0; rr < 2; ++rr)
+        vsc[u][rr] = kPaged ? gvs[g + 8 * rr] : vs_row[min(T + 16 * u + g + 8 * rr, len - 1)];
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
-        const int tok = min(T + 16 * u + 2 * c + (q4 & 1) + 8 * (q4 >> 1), p.Skv - 1);
-        const int8_t* row = vbase + static_cast<size_t>(tok) * row_stride + VB * g;
+        const int off = 2 * c + (q4 & 1) + 8 * (q4 >> 1);
+        const int tok = min(T + 16 * u + off, len - 1);
+        const int8_t* row = (kPaged ? gv + static_cast<size_t>(off) * row_stride
+                                    : vbase + static_cast<size_t>(tok) * row_stride) +
+                            VB * g;
         if constexpr (VB == 16) {
           const uint4 x = ldg_stream16(row);
           vw[u][q4][0] = x.x;
@@ -373,26 +498,64 @@ __global__ void __launch_bounds__(128, FA_DECODE_MIN_CTAS) fa_decode_split_kerne
   }
 }
 
+// One warp per (batch, query head): the lanes read the splits' log-sum-exps together, reduce
+// the maximum and the sum of weights with shuffles, then each lane merges D/32 output dims with
+// vector loads, several splits in flight at once.  Launched as a programmatic dependent of the
+// split kernel: its CTAs may start while the split kernel drains and wait at griddepcontrol.wait
+// until every partial is written and visible.
 template <int D>
-__global__ void __launch_bounds__(D) fa_decode_combine_kernel(const CombineParams p) {
-  const int bh = blockIdx.x;
-  const int d = threadIdx.x;
+__global__ void __launch_bounds__(128) fa_decode_combine_kernel(const CombineParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  constexpr int V = D / 32;  // dims per lane
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int rows = p.B * p.Hq;
+  if (row >= rows) return;
+  const size_t stride = static_cast<size_t>(rows);
   float M = -INFINITY;
-  for (int s = 0; s < p.splits; ++s)
-    M = fmaxf(M, p.lse_part[static_cast<size_t>(s) * p.B * p.Hq + bh]);
-  float L = 0.f, acc = 0.f;
+  for (int s = lane; s < p.splits; s += 32) M = fmaxf(M, p.lse_part[s * stride + row]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float L = 0.f;
+  float acc[V];
+#pragma unroll
+  for (int i = 0; i < V; ++i) acc[i] = 0.f;
   if (M != -INFINITY) {
+    for (int s = lane; s < p.splits; s += 32) {
+      const float ls = p.lse_part[s * stride + row];
+      L += (ls == -INFINITY) ? 0.f : expf(ls - M);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+#pragma unroll 4
     for (int s = 0; s < p.splits; ++s) {
-      const float ls = p.lse_part[static_cast<size_t>(s) * p.B * p.Hq + bh];
-      if (ls == -INFINITY) continue;
-      const float w = expf(ls - M);
-      L += w;
-      acc += w * p.o_part[(static_cast<size_t>(s) * p.B * p.Hq + bh) * D + d];
+      const float ls = p.lse_part[s * stride + row];
+      const float w = (ls == -INFINITY) ? 0.f : expf(ls - M);
+      const float* src = p.o_part + (s * stride + row) * D + V * lane;
+      if constexpr (V == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(src);
+        acc[0] += w * x.x;
+        acc[1 % V] += w * x.y;
+        acc[2 % V] += w * x.z;
+        acc[3 % V] += w * x.w;
+      } else {
+        const float2 x = *reinterpret_cast<const float2*>(src);
+        acc[0] += w * x.x;
+        acc[1 % V] += w * x.y;
+      }
     }
   }
-  const float o = (L > 0.f) ? acc / L : 0.f;
-  p.o[static_cast<size_t>(bh) * D + d] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
-  if (d == 0 && p.lse != nullptr) p.lse[bh] = (L > 0.f) ? M + logf(L) : -INFINITY;
+  const float inv = (L > 0.f) ? 1.f / L : 0.f;
+  uint16_t* dst = p.o + static_cast<size_t>(row) * D + V * lane;
+  if constexpr (V == 4) {
+    uint2 w2;
+    w2.x = pack_bf16x2(acc[0] * inv, acc[1 % V] * inv);
+    w2.y = pack_bf16x2(acc[2 % V] * inv, acc[3 % V] * inv);
+    *reinterpret_cast<uint2*>(dst) = w2;
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1 % V] * inv);
+  }
+  if (lane == 0 && p.lse != nullptr) p.lse[row] = (L > 0.f) ? M + logf(L) : -INFINITY;
 }
 
 }  // namespace fa

@@ -133,10 +133,10 @@ size_t decode_ws_layout(int B, int Hq, int D, int splits, size_t* lse_off) {
   return (off + l_bytes + 255) & ~size_t(255);
 }
 
-template <int D>
-int launch_decode(const void* q, const int8_t* k, const int8_t* v, const float* ks, const float* vs,
-                  void* o, float* lse, int B, int Hq, int Hkv, int Skv, float scale, int splits,
-                  void* ws, cudaStream_t stream) {
+// Fields every decode launch shares; the caller adds the cache addressing.
+fa::DecodeParams decode_params(const void* q, const int8_t* k, const int8_t* v, const float* ks,
+                               const float* vs, int B, int Hq, int Hkv, int D, float scale,
+                               int splits, void* ws) {
   size_t lse_off = 0;
   decode_ws_layout(B, Hq, D, splits, &lse_off);
   fa::DecodeParams p{};
@@ -150,26 +150,68 @@ int launch_decode(const void* q, const int8_t* k, const int8_t* v, const float* 
   p.B = B;
   p.Hq = Hq;
   p.Hkv = Hkv;
-  p.Skv = Skv;
   p.G = Hq / Hkv;
   p.splits = splits;
-  p.chunk = (Skv + splits - 1) / splits;
   p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
-  const long long gz = static_cast<long long>(B) * ((p.G + 7) / 8);
-  if (Hkv > 0x7fffffff || splits > 65535 || gz > 65535) return FA_ERR_INVALID_ARG;
-  dim3 grid(Hkv, splits, static_cast<unsigned>(gz));
-  fa::fa_decode_split_kernel<D><<<grid, 128, 0, stream>>>(p);
+  return p;
+}
+
+// Split kernel over grid (Hkv, splits, B * head blocks), then the merge kernel.
+template <int D, bool kPaged>
+int launch_split_and_combine(const fa::DecodeParams& p, void* o, float* lse, cudaStream_t stream) {
+  const long long gz = static_cast<long long>(p.B) * ((p.G + 7) / 8);
+  if (p.splits > 65535 || gz > 65535) return FA_ERR_INVALID_ARG;
+  dim3 grid(p.Hkv, p.splits, static_cast<unsigned>(gz));
+  fa::fa_decode_split_kernel<D, kPaged><<<grid, 128, 0, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   fa::CombineParams cp{};
   cp.o_part = p.o_part;
   cp.lse_part = p.lse_part;
   cp.o = static_cast<uint16_t*>(o);
   cp.lse = lse;
-  cp.B = B;
-  cp.Hq = Hq;
-  cp.splits = splits;
-  fa::fa_decode_combine_kernel<D><<<B * Hq, D, 0, stream>>>(cp);
+  cp.B = p.B;
+  cp.Hq = p.Hq;
+  cp.splits = p.splits;
+  // The merge is a programmatic dependent launch: its CTAs may be scheduled while the split
+  // kernel drains, and wait on the device (griddepcontrol.wait) for the partials.
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>((static_cast<long long>(p.B) * p.Hq + 3) / 4));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = FA_DECODE_PDL;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, fa::fa_decode_combine_kernel<D>, cp) != cudaSuccess)
+    return FA_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D>
+int launch_decode(const void* q, const int8_t* k, const int8_t* v, const float* ks, const float* vs,
+                  void* o, float* lse, int B, int Hq, int Hkv, int Skv, float scale, int splits,
+                  void* ws, cudaStream_t stream) {
+  fa::DecodeParams p = decode_params(q, k, v, ks, vs, B, Hq, Hkv, D, scale, splits, ws);
+  p.Skv = Skv;
+  p.chunk = (Skv + splits - 1) / splits;
+  return launch_split_and_combine<D, false>(p, o, lse, stream);
+}
+
+template <int D>
+int launch_decode_paged(const void* q, const int8_t* k, const int8_t* v, const float* ks,
+                        const float* vs, const int32_t* block_table, const int32_t* seqlens,
+                        void* o, float* lse, int B, int Hq, int Hkv, int page_shift,
+                        int max_pages, int num_pages, float scale, int splits, void* ws,
+                        cudaStream_t stream) {
+  fa::DecodeParams p = decode_params(q, k, v, ks, vs, B, Hq, Hkv, D, scale, splits, ws);
+  p.block_table = block_table;
+  p.seqlens = seqlens;
+  p.max_pages = max_pages;
+  p.num_pages = num_pages;
+  p.page_shift = page_shift;
+  return launch_split_and_combine<D, true>(p, o, lse, stream);
 }
 
 // Device address of g_noalloc_scratch on the current device.  In host code the symbol name is
@@ -262,6 +304,8 @@ const char* fa_status_string(int status) {
     case FA_ERR_WORKSPACE: return "FA_ERR_WORKSPACE: workspace missing or too small";
     case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA call or kernel launch failed";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a kernel gave up a bounded wait";
+    case FA_ERR_DEVICE_INDEX:
+      return "FA_ERR_DEVICE_INDEX: a page id or sequence length in device memory was out of range";
     default: return "unknown fa_status";
   }
 }
@@ -274,7 +318,8 @@ int fa_device_status(void* stream) {
   const unsigned int zero = 0;
   if (cudaMemcpyToSymbol(fa::g_fa_device_status, &zero, sizeof zero) != cudaSuccess)
     return FA_ERR_CUDA;
-  return (v & fa::kDevStatusTimeout) ? FA_ERR_TIMEOUT : FA_ERR_CUDA;
+  if (v & fa::kDevStatusTimeout) return FA_ERR_TIMEOUT;
+  return (v & fa::kDevStatusBadIndex) ? FA_ERR_DEVICE_INDEX : FA_ERR_CUDA;
 }
 
 int fa_decode_int8_noalloc(const void* q, const int8_t* k, const int8_t* v, const float* k_scale,
@@ -299,6 +344,48 @@ int fa_decode_int8_noalloc(const void* q, const int8_t* k, const int8_t* v, cons
                                        num_splits, ws, s)
                   : launch_decode<64>(q, k, v, k_scale, v_scale, o, lse, B, Hq, Hkv, Skv, scale,
                                       num_splits, ws, s);
+}
+
+int fa_decode_int8_paged(const void* q, const int8_t* k_pages, const int8_t* v_pages,
+                         const float* k_scale_pages, const float* v_scale_pages,
+                         const int32_t* block_table, const int32_t* seqlens, void* o, float* lse,
+                         int B, int Hq, int Hkv, int page_size, int max_pages_per_seq,
+                         int num_pages, int D, float scale, int num_splits, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  if (!q || !k_pages || !v_pages || !k_scale_pages || !v_scale_pages || !block_table ||
+      !seqlens || !o)
+    return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || num_splits <= 0 || max_pages_per_seq <= 0 ||
+      num_pages <= 0)
+    return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  int page_shift = -1;
+  for (int s = 4; s <= 16; ++s)
+    if (page_size == (1 << s)) page_shift = s;
+  if (page_shift < 0) return FA_ERR_INVALID_ARG;
+  if ((static_cast<long long>(max_pages_per_seq) << page_shift) > (1ll << 30))
+    return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) ||
+      !aligned16(k_scale_pages) || !aligned16(v_scale_pages) ||
+      (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+      (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FA_ERR_ALIGNMENT;
+  const size_t need = decode_ws_layout(B, Hq, D, num_splits, nullptr);
+  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_ALIGNMENT;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return D == 128
+             ? launch_decode_paged<128>(q, k_pages, v_pages, k_scale_pages, v_scale_pages,
+                                        block_table, seqlens, o, lse, B, Hq, Hkv, page_shift,
+                                        max_pages_per_seq, num_pages, scale, num_splits,
+                                        workspace, st)
+             : launch_decode_paged<64>(q, k_pages, v_pages, k_scale_pages, v_scale_pages,
+                                       block_table, seqlens, o, lse, B, Hq, Hkv, page_shift,
+                                       max_pages_per_seq, num_pages, scale, num_splits,
+                                       workspace, st);
 }
 
 int fa_selftest_bounded_wait(int timeout_us, void* stream) {

@@ -11,10 +11,11 @@
 
 namespace fa {
 
-// Device-side status word.  Kernels OR these bits in when a bounded wait gives up; the host
-// reads and clears it in fa_device_status().  The library is built as a single translation
-// unit, so the definition lives here.
-enum : unsigned { kDevStatusTimeout = 1u };
+// Device-side status word.  Kernels OR these bits in when a bounded wait gives up, or when an
+// index read from device memory (a page id, a sequence length) is out of range; the host reads
+// and clears it in fa_device_status().  The library is built as a single translation unit, so
+// the definition lives here.
+enum : unsigned { kDevStatusTimeout = 1u, kDevStatusBadIndex = 2u };
 __device__ unsigned int g_fa_device_status = 0;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
