@@ -98,7 +98,8 @@ FA_API size_t fa_decode_int8_workspace_bytes(int B, int Hq, int D, int num_split
  *   k_scale, v_scale fp32 [B, Hkv, Skv]
  *   o       bf16 [B, 1, Hq, D]     written
  *   lse     fp32 [B, Hq] natural log, or NULL
- *   num_splits >= 1: the keys are cut into chunks of ceil(Skv / num_splits); each chunk is
+ *   num_splits >= 1: the keys are cut into chunks of ceil(Skv / num_splits) keys rounded up to
+ *           a multiple of 128 (so fewer chunks than num_splits may hold keys); each chunk is
  *           reduced to a partial (output, log-sum-exp) in `workspace`, and a second kernel
  *           merges the partials through their log-sum-exp.
  *   workspace  device buffer of at least fa_decode_int8_workspace_bytes(B, Hq, D, num_splits)
@@ -161,9 +162,9 @@ FA_API int fa_decode_int8_noalloc(const void* q, const int8_t* k, const int8_t* 
  *   o, lse   as for fa_decode_int8.
  *   page_size  a power of two, 16 .. 65536; max_pages_per_seq * page_size <= 2^30.
  *   num_pages  number of pages in the pool (page ids are 0 .. num_pages - 1).
- *   num_splits >= 1: each sequence's keys are cut into num_splits chunks of
- *            ceil(seqlens[b] / num_splits) keys rounded up to a multiple of 16; chunks are
- *            merged through their log-sum-exp as in fa_decode_int8.
+ *   num_splits >= 1: each sequence's keys are cut into chunks of ceil(seqlens[b] / num_splits)
+ *            keys rounded up to a multiple of 128 (a short sequence fills only its first
+ *            chunks); chunks are merged through their log-sum-exp as in fa_decode_int8.
  *   workspace  at least fa_decode_int8_workspace_bytes(B, Hq, D, num_splits) bytes.
  * block_table and seqlens need 4-byte alignment; every other tensor 16-byte alignment.
  * The lengths and page ids live in device memory, so they are checked on the device: an id

@@ -8,29 +8,36 @@
 // so the scales leave the dot products and each code converts exactly to fp16.
 //
 // Split step (fa_decode_split_kernel): one CTA per (split, batch, KV head, block of <= 8 query
-// heads of that KV head's group); 4 warps stride over the split's keys 32 at a time.  Each warp
-// streams the int8 rows straight from HBM into registers with 16-byte non-caching loads,
-// converts them to fp16 with byte permutes and one fp16 subtract, and runs both contractions on
-// the tensor cores with mma.sync m16n8k16 (fp32 accumulate):
-//   S  = Kcode[16 tokens x 16 dims] . Q^T[16 dims x 8 heads]   (tokens as M, heads as N)
-//   O^T += Vcode^T[16 dims x 16 tokens] . P'^T[16 tokens x 8 heads]
+// heads of that KV head's group).  A producer warp streams the split's keys into a ring of
+// shared-memory stages of 128 keys: the int8 K and V rows by TMA tensor copies (the codes never
+// pass through registers on their way in, so the bytes in flight are bounded by shared memory,
+// not by the register file), their fp32 scales by 4-byte asynchronous copies, all completing on
+// one mbarrier per stage.  Four consumer warps each take 32 keys of every stage, read the rows
+// in their MMA fragment layout, convert the codes to fp16 with byte permutes and one fp16
+// subtract, and run both contractions on the tensor cores with mma.sync m16n8k16 (fp32
+// accumulate):
+//   S  = Kcode[16 keys x 16 dims] . Q^T[16 dims x 8 heads]   (keys as M, heads as N)
+//   O^T += Vcode^T[16 dims x 16 keys] . P'^T[16 keys x 8 heads]
 // The reduction index of each contraction is permuted (dims for QK, dims of the output rows
 // for PV) so that every thread's fragment comes from contiguous bytes of one row; Q and the
-// output use the same permutations, so the results are unchanged.  P' = p * v_scale is moved
-// from the QK accumulator layout into the PV operand layout with movmatrix (8x8 transpose).
-// The online softmax (running max m and sum l per head, rescale when m grows by more than 2^8)
-// runs on the accumulator fragments.  The 4 warps merge through shared memory and the CTA
-// writes a normalised partial output and its log-sum-exp to the workspace.
+// output use the same permutations, so the results are unchanged.  P' = p * v_scale * 2^E is
+// moved from the QK accumulator layout into the PV operand layout with movmatrix (8x8
+// transpose); E keeps P' inside the fp16 range and is lowered, with an exact power-of-two
+// rescale of the accumulator, whenever a larger v_scale arrives.  The online softmax (running
+// max m and sum l per head, rescale when m grows by more than 2^8) runs on the accumulator
+// fragments.  The 4 warps merge through shared memory and the CTA writes a normalised partial
+// output and its log-sum-exp to the workspace.
 //
-// Paged variant (kPaged): the cache is a pool of pages of P tokens (P a power of two >= 16),
+// Paged variant (kPaged): the cache is a pool of pages of P keys (P a power of two >= 16),
 // [num_pages, P, Hkv, D] codes and [num_pages, Hkv, P] scales, and sequence b owns the pages
 // listed in block_table[b] ("Sparse attention and MLA operators in ops-transformer", section 2.2:
 // the KV cache addressed through a block_table) and has its own length seqlens[b], read on the
 // device ("Flash Attention on Ascend: three techniques", version section: sequences of different
-// lengths in one batch).  Each split covers ceil(len / splits) keys rounded up to 16, so every
-// 16-token group of a step lies inside one page: the page is looked up once per group.  Page ids
-// and lengths are range-checked; a bad one is recorded in the device status word and replaced by
-// a valid one, so a corrupt table never makes the kernel read outside the pool.
+// lengths in one batch).  The page becomes a TMA coordinate: a stage is min(128, P)-key boxes at
+// (row in page, page id).  Splits are whole stages (ceil(len / splits) rounded up to 128 keys),
+// so short sequences occupy few splits and the rest exit at once.  Page ids and lengths are
+// range-checked; a bad one is recorded in the device status word and replaced by a valid one,
+// so a corrupt table never makes the kernel read outside the pool.
 //
 // Merge step (fa_decode_combine_kernel): L = log sum_s exp(L_s), O = sum_s exp(L_s - L) O_s.
 #pragma once
@@ -47,7 +54,7 @@ struct DecodeParams {
   const float* v_scale;
   float* o_part;    // [splits, B, Hq, D]
   float* lse_part;  // [splits, B, Hq]
-  int B, Hq, Hkv, Skv, G, splits, chunk;
+  int B, Hq, Hkv, Skv, G, splits;
   float scale_log2;
   // paged cache only
   const int32_t* block_table;  // [B, max_pages]
@@ -62,22 +69,6 @@ struct CombineParams {
   float* lse;   // [B, Hq] or null
   int B, Hq, splits;
 };
-
-__device__ __forceinline__ uint4 ldg_stream16(const void* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
-
-__device__ __forceinline__ uint2 ldg_stream8(const void* p) {
-  uint2 r;
-  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
-               : "=r"(r.x), "=r"(r.y)
-               : "l"(p));
-  return r;
-}
 
 // Two biased bytes (x + 128) in the low bytes of a fp16 pair with exponent 2^10 give
 // 1024 + x + 128 exactly; subtracting 1152 leaves x exactly.
@@ -123,38 +114,112 @@ __device__ __forceinline__ int pow2_exponent_below(float x, int top) {
 
 __device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) << 23); }
 
-#ifndef FA_PAGED_SMEM_PAGES
-#define FA_PAGED_SMEM_PAGES 1  // stage each split's page ids in shared memory
-#endif
+__device__ __forceinline__ float exp2i_or_zero(int e) { return e < -126 ? 0.f : exp2i(e); }
 
-#ifndef FA_PAGED_VMAX_BATCH
-#define FA_PAGED_VMAX_BATCH 1
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 r;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "r"(addr));
+  return r;
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+  uint2 r;
+  asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
+  return r;
+}
+
+__device__ __forceinline__ float lds32f(uint32_t addr) {
+  float r;
+  asm volatile("ld.shared.f32 %0, [%1];" : "=f"(r) : "r"(addr));
+  return r;
+}
+
+// 4-byte asynchronous global -> shared copy, and the mbarrier arrival that fires once every
+// such copy of this thread has landed (the arrival raises the barrier's pending count when it
+// is issued, so the phase cannot complete before the copies do).
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+#ifndef FA_DECODE_STAGES
+#define FA_DECODE_STAGES 2  // K/V stages of 128 keys in the shared-memory ring (3 CTAs per SM)
 #endif
 
 #ifndef FA_DECODE_PDL
 #define FA_DECODE_PDL 1  // launch the merge kernel as a programmatic dependent of the split kernel
 #endif
 
-#ifndef FA_DECODE_MIN_CTAS
-#define FA_DECODE_MIN_CTAS 3  // CTAs per SM the register allocation must allow
-#endif
+// Shared-memory plan of the split kernel.  A stage holds 128 keys: the K and V code tiles
+// ([128 rows][D bytes], 128B-swizzled for D = 128 so that the row-per-lane fragment reads are
+// conflict free) and their fp32 scales.
+template <int D>
+struct DecodeCfg {
+  static constexpr int kT = 128;                  // keys per stage
+  static constexpr int kStages = FA_DECODE_STAGES;
+  static constexpr int kTile = kT * D;            // bytes of one K or V code tile
+  static constexpr int kStageBytes = 2 * kTile;
+  static constexpr int kScaleOff = kStages * kStageBytes;  // fp32 [stages][K, V][kT]
+  static constexpr int kBarOff = kScaleOff + kStages * 2 * kT * 4;
+  static constexpr int kMiscOff = kBarOff + 16 * kStages;  // abort flag
+  static constexpr int kPageStage = 256;                   // page ids staged per split
+  static constexpr int kPageOff = kMiscOff + 16;
+  static constexpr int kEnd = kPageOff + 4 * kPageStage;
+  static constexpr int kSmemBytes = kEnd + 1024;           // + alignment of the dynamic base
+  static constexpr bool kSwizzle = (D == 128);
+  // merge buffers, reused from the stage tiles once the key loop is over
+  static constexpr int kMergeO = 0;                        // fp32 [4 warps][8 heads][D]
+  static constexpr int kMergeM = 4 * 8 * D * 4;            // fp32 [4][8]
+  static constexpr int kMergeL = kMergeM + 4 * 8 * 4;      // fp32 [4][8]
+  static_assert(kMergeL + 4 * 8 * 4 <= kScaleOff, "merge buffers must fit in the stage tiles");
+};
+
+// Byte offset of 16-byte chunk `chunk` of row `row` in a code tile whose base is 1024-aligned.
+template <int D>
+__device__ __forceinline__ uint32_t tile_off(int row, int chunk) {
+  if constexpr (D == 128) return row * 128 + ((chunk ^ (row & 7)) << 4);
+  else return row * D + (chunk << 4);
+}
 
 template <int D, bool kPaged>
-__global__ void __launch_bounds__(128, FA_DECODE_MIN_CTAS) fa_decode_split_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(160, 1) fa_decode_split_kernel(
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+    const DecodeParams p) {
+  using C = DecodeCfg<D>;
   constexpr int KS = D / 16;  // QK k-steps
   constexpr int MT = D / 16;  // PV m-tiles (16 output dims each)
-  constexpr int VB = D / 8;   // V bytes per thread per token
-  // grid (Hkv, splits, B * head blocks): the KV head varies fastest, so CTAs running at the
-  // same time stream the same token rows (all KV heads of a token are contiguous in memory).
+  constexpr int VB = D / 8;   // V bytes per thread per key
+  constexpr int QB = D / 4;   // K bytes per thread per key (its share of the dims)
   // the merge kernel may be scheduled as soon as every CTA of this grid has started
   asm volatile("griddepcontrol.launch_dependents;");
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sb = smem_u32(smem);
+  auto bar_full = [&](int s) { return sb + C::kBarOff + 8 * s; };
+  auto bar_empty = [&](int s) { return sb + C::kBarOff + 8 * (C::kStages + s); };
+  int* abort_flag = reinterpret_cast<int*>(smem + C::kMiscOff);
+  int* sm_pages = reinterpret_cast<int*>(smem + C::kPageOff);
+  const WaitCtl ctl{abort_flag, 4000000000ull};
+
+  // grid (Hkv, splits, B * head blocks): the KV head varies fastest, so CTAs running at the
+  // same time stream the same key rows (all KV heads of a key are contiguous in memory).
   const int kvh = blockIdx.x, split = blockIdx.y;
   const int nhb = (p.G + 7) / 8;
   const int b = static_cast<int>(blockIdx.z) / nhb, hb = static_cast<int>(blockIdx.z) % nhb;
   const int head0 = kvh * p.G + hb * 8;
   const int nheads = min(8, p.G - hb * 8);
-  int len = p.Skv, chunk = p.chunk;
-  const int32_t* bt_row = nullptr;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  int len = p.Skv;
   if constexpr (kPaged) {
     const int cap = p.max_pages << p.page_shift;
     len = p.seqlens[b];
@@ -162,107 +227,119 @@ __global__ void __launch_bounds__(128, FA_DECODE_MIN_CTAS) fa_decode_split_kerne
       if (threadIdx.x == 0) atomicOr(&g_fa_device_status, kDevStatusBadIndex);
       len = max(0, min(len, cap));
     }
-    chunk = ((len + p.splits - 1) / p.splits + 15) & ~15;
-    bt_row = p.block_table + static_cast<size_t>(b) * p.max_pages;
   }
-  const int t_begin = split * chunk;
+  // splits are whole stages: every stage starts on a multiple of 128 keys
+  const int chunk = ((len + p.splits - 1) / p.splits + C::kT - 1) / C::kT * C::kT;
+  const int t_begin = min(len, split * chunk);
   const int t_end = min(len, t_begin + chunk);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_stages = (t_end - t_begin + C::kT - 1) / C::kT;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_empty(s), 4);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == 4) {
+    // ============================ producer warp ============================
+    const int pmask = (1 << p.page_shift) - 1;
+    const int32_t* bt_row = kPaged ? p.block_table + static_cast<size_t>(b) * p.max_pages : nullptr;
+    auto checked_page = [&](int slot) -> int {
+      int pg = bt_row[slot];
+      if (static_cast<unsigned>(pg) >= static_cast<unsigned>(p.num_pages)) {
+        atomicOr(&g_fa_device_status, kDevStatusBadIndex);
+        pg = 0;
+      }
+      return pg;
+    };
+    const int first_slot = kPaged ? (t_begin >> p.page_shift) : 0;
+    const int n_slots = (kPaged && n_stages > 0) ? ((t_end - 1) >> p.page_shift) - first_slot + 1 : 0;
+    const bool staged = n_slots <= C::kPageStage;
+    if constexpr (kPaged) {
+      if (staged)
+        for (int i = lane; i < n_slots; i += 32) sm_pages[i] = checked_page(first_slot + i);
+      __syncwarp();
+    }
+    // page of key t (t_begin <= t < t_end)
+    auto page_of = [&](int t) -> int {
+      const int slot = t >> p.page_shift;
+      return staged ? sm_pages[slot - first_slot] : checked_page(slot);
+    };
+    const int box_t = kPaged ? min(C::kT, 1 << p.page_shift) : C::kT;  // keys per TMA box
+    const float* ks_row = p.k_scale + (static_cast<size_t>(b) * p.Hkv + kvh) * p.Skv;
+    const float* vs_row = p.v_scale + (static_cast<size_t>(b) * p.Hkv + kvh) * p.Skv;
+
+    int issued = 0;
+    for (int i = 0; i < n_stages; ++i) {
+      const int s = i % C::kStages;
+      if (i >= C::kStages && !mbar_wait(bar_empty(s), ((i / C::kStages) - 1) & 1, ctl)) break;
+      const int t0 = t_begin + C::kT * i;
+      // scales of the stage's keys: 4-byte asynchronous copies, 4 keys per lane
+      const uint32_t ks_dst = sb + C::kScaleOff + s * 2 * C::kT * 4;
+      const uint32_t vs_dst = ks_dst + C::kT * 4;
+#pragma unroll
+      for (int j = 0; j < C::kT / 32; ++j) {
+        const int r = lane + 32 * j, t = t0 + r;
+        if (t < t_end) {
+          const float *ksrc, *vsrc;
+          if constexpr (kPaged) {
+            const size_t idx =
+                ((static_cast<size_t>(page_of(t)) * p.Hkv + kvh) << p.page_shift) + (t & pmask);
+            ksrc = p.k_scale + idx;
+            vsrc = p.v_scale + idx;
+          } else {
+            ksrc = ks_row + t;
+            vsrc = vs_row + t;
+          }
+          cp_async4(ks_dst + 4 * r, ksrc);
+          cp_async4(vs_dst + 4 * r, vsrc);
+        }
+      }
+      cp_async_mbar_arrive(bar_full(s));
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar_full(s), C::kStageBytes);
+        const uint32_t kt = sb + s * C::kStageBytes, vt = kt + C::kTile;
+        for (int t = t0; t < t0 + C::kT; t += box_t) {
+          const uint32_t off = (t - t0) * D;
+          if constexpr (kPaged) {
+            // a box past the split's last key reads the split's last page (its keys are masked)
+            const int pg = page_of(min(t, t_end - 1));
+            const int r0 = t & pmask;
+            tma_load_4d(kt + off, &tm_k, bar_full(s), 0, kvh, r0, pg);
+            tma_load_4d(vt + off, &tm_v, bar_full(s), 0, kvh, r0, pg);
+          } else {
+            tma_load_4d(kt + off, &tm_k, bar_full(s), 0, kvh, t, b);
+            tma_load_4d(vt + off, &tm_v, bar_full(s), 0, kvh, t, b);
+          }
+        }
+      }
+      issued = i + 1;
+    }
+    // Every copy this warp started has landed before the CTA can exit (already true on the
+    // normal path; after a consumer gave up this waits, bounded, for copies in flight).
+    cp_async_wait_all();
+    if (lane == 0) {
+      volatile int zero = 0;
+      const WaitCtl drain_ctl{&zero, 4000000000ull};
+      for (int s = 0; s < C::kStages && s < issued; ++s) {
+        const int last = s + C::kStages * ((issued - 1 - s) / C::kStages);
+        mbar_wait(bar_full(s), (last / C::kStages) & 1, drain_ctl);
+      }
+    }
+    return;
+  }
+
+  // ============================ consumer warps 0..3 ============================
   const int g = lane >> 2, c = lane & 3;
 
-  __shared__ float sm_red[4];
-  __shared__ float sm_m[4][8], sm_l[4][8];
-  __shared__ float sm_o[4][8][D];
-
-  const size_t row_stride = static_cast<size_t>(p.Hkv) * D;  // bytes between tokens
-  const int pmask = (1 << p.page_shift) - 1;
-  // physical page of key t (t < len): checked against the pool, never outside it
-  auto checked_page = [&](int slot) -> int {
-    int pg = bt_row[slot];
-    if (static_cast<unsigned>(pg) >= static_cast<unsigned>(p.num_pages)) {
-      atomicOr(&g_fa_device_status, kDevStatusBadIndex);
-      pg = 0;
-    }
-    return pg;
-  };
-#if FA_PAGED_SMEM_PAGES
-  // The split's page ids are staged in shared memory once (checked there), so the loads of a
-  // step never wait on a dependent global load.  A split spanning more pages than the stage
-  // holds reads the table directly.
-  constexpr int kPageStage = 512;
-  __shared__ int sm_pages[kPageStage];
-  const int first_slot = kPaged ? (t_begin >> p.page_shift) : 0;
-  const int n_slots = (kPaged && t_end > t_begin) ? ((t_end - 1) >> p.page_shift) - first_slot + 1 : 0;
-  const bool staged = n_slots <= kPageStage;
-  if constexpr (kPaged) {
-    if (staged)
-      for (int i = threadIdx.x; i < n_slots; i += 128) sm_pages[i] = checked_page(first_slot + i);
-    __syncthreads();
-  }
-  auto page_of = [&](int t) -> int {
-    const int slot = t >> p.page_shift;
-    return staged ? sm_pages[slot - first_slot] : checked_page(slot);
-  };
-#else
-  auto page_of = [&](int t) -> int { return checked_page(t >> p.page_shift); };
-#endif
-  // offset of (page pg, kv head kvh, row r) in the [num_pages, Hkv, P] scale arrays
-  auto page_scale_index = [&](int pg, int r) -> size_t {
-    return ((static_cast<size_t>(pg) * p.Hkv + kvh) << p.page_shift) + r;
-  };
-  // paged: code row and scale pointers of the 16-token group that starts at key gs0.  A group
-  // past the split's last key is replaced by the split's last group (its extra keys are masked),
-  // so every page looked up belongs to this split.
-  const int last16 = (t_end - 1) & ~15;
-  auto group_base = [&](int gs0, const int8_t* codes, const float* scales, const int8_t*& rows,
-                        const float*& sc) {
-    const int gs = min(gs0, last16);
-    const int pg = page_of(gs);
-    const int r0 = gs & pmask;
-    rows = codes + ((static_cast<size_t>(pg) << p.page_shift) + r0) * row_stride +
-           static_cast<size_t>(kvh) * D;
-    sc = scales + page_scale_index(pg, r0);
-  };
-
-  const float* ks_row = p.k_scale + (static_cast<size_t>(b) * p.Hkv + kvh) * p.Skv;
-  const float* vs_row = p.v_scale + (static_cast<size_t>(b) * p.Hkv + kvh) * p.Skv;
-
-  // ---- P' = p * v_scale * 2^E stays below 2^15 in fp16: E from the split's largest v_scale ----
-  float vmax = 0.f;
-  if constexpr (kPaged) {
-#if FA_PAGED_VMAX_BATCH
-    // 8 keys per thread per round: all page ids, then all scales, so each round waits for two
-    // memory latencies instead of sixteen
-    for (int t0 = t_begin + threadIdx.x; t0 < t_end; t0 += 128 * 8) {
-      int pg[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int t = min(t0 + 128 * i, t_end - 1);
-        pg[i] = page_of(t);
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int t = t0 + 128 * i;
-        const float sv = p.v_scale[page_scale_index(pg[i], min(t, t_end - 1) & pmask)];
-        vmax = fmaxf(vmax, sv);
-      }
-    }
-#else
-    for (int t = t_begin + threadIdx.x; t < t_end; t += 128)
-      vmax = fmaxf(vmax, p.v_scale[page_scale_index(page_of(t), t & pmask)]);
-#endif
-  } else {
-    for (int t = t_begin + threadIdx.x; t < t_end; t += 128) vmax = fmaxf(vmax, vs_row[t]);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
-  if (lane == 0) sm_red[warp] = vmax;
-  __syncthreads();
-  vmax = fmaxf(fmaxf(sm_red[0], sm_red[1]), fmaxf(sm_red[2], sm_red[3]));
-  const int E = pow2_exponent_below(vmax, 7);  // p <= 2^8 with the lazy rescale
-  const float pscale = exp2i(E);
-
   // ---- Q as the B operand of the QK mma, fp16, scaled by 2^eq per head (exact) ----
+  // Thread c holds dims [QB*c, QB*c + QB) of its head: k-step s, element e is dim QB*c + 4s + e,
+  // the same dims its K fragment reads from each key row.
   uint32_t qf[KS][2];
   float sc_mine;
   {
@@ -274,8 +351,7 @@ __global__ void __launch_bounds__(128, FA_DECODE_MIN_CTAS) fa_decode_split_kerne
     for (int s = 0; s < KS; ++s)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int dim = (s / 4) * 64 + 16 * c + 4 * (s % 4) + e;
-        qv[s][e] = hv ? bf16_bits_to_float(qrow[dim]) : 0.f;
+        qv[s][e] = hv ? bf16_bits_to_float(qrow[QB * c + 4 * s + e]) : 0.f;
         amax = fmaxf(amax, fabsf(qv[s][e]));
       }
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
@@ -297,203 +373,206 @@ __global__ void __launch_bounds__(128, FA_DECODE_MIN_CTAS) fa_decode_split_kerne
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) oacc[mt][0] = oacc[mt][1] = oacc[mt][2] = oacc[mt][3] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  // P' = p * v_scale * 2^E must stay below 2^15 in fp16 (p <= 2^8 with the lazy rescale): the
+  // warp lowers E, rescaling its output accumulator, whenever a larger v_scale arrives.
+  constexpr int kEUnset = 1 << 20;
+  int E = kEUnset;
 
-  const int8_t* kbase = p.k + (static_cast<size_t>(b) * p.Skv * p.Hkv + kvh) * D;
-  const int8_t* vbase = p.v + (static_cast<size_t>(b) * p.Skv * p.Hkv + kvh) * D;
-  const int nsteps = (t_end - t_begin + 31) / 32;
+  for (int i = 0; i < n_stages; ++i) {
+    const int s = i % C::kStages;
+    if (!mbar_wait(bar_full(s), (i / C::kStages) & 1, ctl)) break;
+    const int T = t_begin + C::kT * i + 32 * warp;  // this warp's 32 keys of the stage
+    if (T < t_end) {
+      const uint32_t kt = sb + s * C::kStageBytes, vt = kt + C::kTile;
+      const uint32_t ks_s = sb + C::kScaleOff + s * 2 * C::kT * 4, vs_s = ks_s + C::kT * 4;
+      const int r_w = 32 * warp;  // first row of this warp in the stage tiles
 
-  // Each warp takes every 4th 32-token step.  Loads run one step ahead without extra registers:
-  // the next step's K rows are requested as soon as this step's QK^T has consumed the K
-  // registers, the next step's V rows as soon as PV has consumed the V registers.
-  uint32_t kw[2][2][KS];  // [group][row g / g+8][k-step]
-  uint32_t vw[2][4][VB / 4];
-  float ksc[2][2], vsc[2][2];
-  auto load_k = [&](int T) {
+      // -- S = Kcode . Q^T per 16-key group; x = score in log2 units --
+      float x[2][4];
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int8_t* gk = nullptr;
-      const float* gks = nullptr;
-      if constexpr (kPaged) group_base(T + 16 * u, p.k, p.k_scale, gk, gks);
+      for (int u = 0; u < 2; ++u) {
+        uint32_t kw[2][KS];
 #pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int tok = min(T + 16 * u + g + 8 * rr, len - 1);
-        const int8_t* row = kPaged ? gk + static_cast<size_t>(g + 8 * rr) * row_stride
-                                   : kbase + static_cast<size_t>(tok) * row_stride;
-        const uint4 lo = ldg_stream16(row + 16 * c);
-        kw[u][rr][0] = lo.x;
-        kw[u][rr][1] = lo.y;
-        kw[u][rr][2] = lo.z;
-        kw[u][rr][3] = lo.w;
-        if constexpr (D == 128) {
-          const uint4 hi = ldg_stream16(row + 64 + 16 * c);
-          kw[u][rr][4 % KS] = hi.x;
-          kw[u][rr][5 % KS] = hi.y;
-          kw[u][rr][6 % KS] = hi.z;
-          kw[u][rr][7 % KS] = hi.w;
+        for (int rr = 0; rr < 2; ++rr) {
+          const int row = r_w + 16 * u + g + 8 * rr;
+          if constexpr (D == 128) {
+            const uint4 lo = lds128(kt + tile_off<D>(row, 2 * c));
+            const uint4 hi = lds128(kt + tile_off<D>(row, 2 * c + 1));
+            kw[rr][0] = lo.x; kw[rr][1] = lo.y; kw[rr][2] = lo.z; kw[rr][3] = lo.w;
+            kw[rr][4 % KS] = hi.x; kw[rr][5 % KS] = hi.y; kw[rr][6 % KS] = hi.z; kw[rr][7 % KS] = hi.w;
+          } else {
+            const uint4 lo = lds128(kt + tile_off<D>(row, c));
+            kw[rr][0] = lo.x; kw[rr][1] = lo.y; kw[rr][2 % KS] = lo.z; kw[rr][3 % KS] = lo.w;
+          }
         }
-        ksc[u][rr] = kPaged ? gks[g + 8 * rr] : ks_row[tok];
+        float sacc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int st = 0; st < KS; ++st) {
+          const uint32_t w0 = kw[0][st] ^ 0x80808080u, w1 = kw[1][st] ^ 0x80808080u;
+          mma_f16_16816(sacc, codes_to_f16x2(w0, kSelB01), codes_to_f16x2(w1, kSelB01),
+                        codes_to_f16x2(w0, kSelB23), codes_to_f16x2(w1, kSelB23), qf[st][0],
+                        qf[st][1]);
+        }
+        const int rA = r_w + 16 * u + g, rB = rA + 8;
+        const int tA = T + 16 * u + g, tB = tA + 8;
+        const float kA = lds32f(ks_s + 4 * rA), kB = lds32f(ks_s + 4 * rB);
+        x[u][0] = tA < t_end ? sacc[0] * kA * sc0 : -INFINITY;
+        x[u][1] = tA < t_end ? sacc[1] * kA * sc1 : -INFINITY;
+        x[u][2] = tB < t_end ? sacc[2] * kB * sc0 : -INFINITY;
+        x[u][3] = tB < t_end ? sacc[3] * kB * sc1 : -INFINITY;
       }
-    }
-  };
-  auto load_v = [&](int T) {
+
+      // -- online softmax per head (columns 2c, 2c+1); max over the warp's 32 keys --
+      float mx0 = fmaxf(fmaxf(x[0][0], x[0][2]), fmaxf(x[1][0], x[1][2]));
+      float mx1 = fmaxf(fmaxf(x[0][1], x[0][3]), fmaxf(x[1][1], x[1][3]));
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int8_t* gv = nullptr;
-      const float* gvs = nullptr;
-      if constexpr (kPaged) group_base(T + 16 * u, p.v, p.v_scale, gv, gvs);
+      for (int o = 4; o < 32; o <<= 1) {
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+      }
+      if (mx0 > m0 + 8.f) {
+        const float a = ex2(m0 - mx0);
+        m0 = mx0;
+        l0 *= a;
 #pragma unroll
-      for (int rr = 0; rr < 2; ++rr)
-        vsc[u][rr] = kPaged ? gvs[g + 8 * rr] : vs_row[min(T + 16 * u + g + 8 * rr, len - 1)];
+        for (int mt = 0; mt < MT; ++mt) {
+          oacc[mt][0] *= a;
+          oacc[mt][2] *= a;
+        }
+      }
+      if (mx1 > m1 + 8.f) {
+        const float a = ex2(m1 - mx1);
+        m1 = mx1;
+        l1 *= a;
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        const int off = 2 * c + (q4 & 1) + 8 * (q4 >> 1);
-        const int tok = min(T + 16 * u + off, len - 1);
-        const int8_t* row = (kPaged ? gv + static_cast<size_t>(off) * row_stride
-                                    : vbase + static_cast<size_t>(tok) * row_stride) +
-                            VB * g;
-        if constexpr (VB == 16) {
-          const uint4 x = ldg_stream16(row);
-          vw[u][q4][0] = x.x;
-          vw[u][q4][1 % (VB / 4)] = x.y;
-          vw[u][q4][2 % (VB / 4)] = x.z;
-          vw[u][q4][3 % (VB / 4)] = x.w;
-        } else {
-          const uint2 x = ldg_stream8(row);
-          vw[u][q4][0] = x.x;
-          vw[u][q4][1 % (VB / 4)] = x.y;
+        for (int mt = 0; mt < MT; ++mt) {
+          oacc[mt][1] *= a;
+          oacc[mt][3] *= a;
+        }
+      }
+      const float mu0 = (m0 == -INFINITY) ? 0.f : m0;
+      const float mu1 = (m1 == -INFINITY) ? 0.f : m1;
+
+      // -- value scales of the warp's keys; lower E if a larger one arrived --
+      float vsc[2][2];
+      float vmax = 0.f;
+#pragma unroll
+      for (int u = 0; u < 2; ++u)
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const int row = r_w + 16 * u + g + 8 * rr;
+          vsc[u][rr] = (T + 16 * u + g + 8 * rr < t_end) ? lds32f(vs_s + 4 * row) : 0.f;
+          vmax = fmaxf(vmax, vsc[u][rr]);
+        }
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+      const int e_step = pow2_exponent_below(vmax, 7);
+      if (e_step < E) {
+        if (E != kEUnset) {
+          const float a = exp2i_or_zero(e_step - E);
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            oacc[mt][0] *= a;
+            oacc[mt][1] *= a;
+            oacc[mt][2] *= a;
+            oacc[mt][3] *= a;
+          }
+        }
+        E = e_step;
+      }
+      const float pscale = exp2i(E);
+
+      uint32_t pb[2][2];  // PV B operand per group: keys 0-7 and 8-15 of the group
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const float pa0 = ex2(x[u][0] - mu0), pa1 = ex2(x[u][1] - mu1);
+        const float pb0 = ex2(x[u][2] - mu0), pb1 = ex2(x[u][3] - mu1);
+        l0 += pa0 + pb0;
+        l1 += pa1 + pb1;
+        const float wa = vsc[u][0] * pscale, wb = vsc[u][1] * pscale;
+        pb[u][0] = movmatrix_trans(pack_f16x2(pa0 * wa, pa1 * wa));
+        pb[u][1] = movmatrix_trans(pack_f16x2(pb0 * wb, pb1 * wb));
+      }
+
+      // -- O^T += Vcode^T . P'^T --
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        uint32_t r[4][VB / 4];
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const int row = r_w + 16 * u + 2 * c + (q4 & 1) + 8 * (q4 >> 1);
+          if constexpr (VB == 16) {
+            const uint4 v4 = lds128(vt + tile_off<D>(row, g));
+            r[q4][0] = v4.x ^ 0x80808080u;
+            r[q4][1 % (VB / 4)] = v4.y ^ 0x80808080u;
+            r[q4][2 % (VB / 4)] = v4.z ^ 0x80808080u;
+            r[q4][3 % (VB / 4)] = v4.w ^ 0x80808080u;
+          } else {
+            const uint2 v2 = lds64(vt + row * D + VB * g);
+            r[q4][0] = v2.x ^ 0x80808080u;
+            r[q4][1 % (VB / 4)] = v2.y ^ 0x80808080u;
+          }
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          const int w = mt >> 1;
+          const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
+          const uint32_t x01 = prmt(r[0][w], r[1][w], sel);  // keys 2c, 2c+1
+          const uint32_t x89 = prmt(r[2][w], r[3][w], sel);  // keys 2c+8, 2c+9
+          mma_f16_16816(oacc[mt], codes_to_f16x2(x01, kSelB01), codes_to_f16x2(x01, kSelB23),
+                        codes_to_f16x2(x89, kSelB01), codes_to_f16x2(x89, kSelB23), pb[u][0],
+                        pb[u][1]);
         }
       }
     }
-  };
-  if (warp < nsteps) {
-    load_k(t_begin + 32 * warp);
-    load_v(t_begin + 32 * warp);
-  }
-  for (int st = warp; st < nsteps; st += 4) {
-    const int T = t_begin + 32 * st;
-    const bool has_next = st + 4 < nsteps;
-
-    // -- S = Kcode . Q^T per 16-token group; x = score in log2 units --
-    float x[2][4];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      float sacc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int s = 0; s < KS; ++s) {
-        const uint32_t w0 = kw[u][0][s] ^ 0x80808080u, w1 = kw[u][1][s] ^ 0x80808080u;
-        mma_f16_16816(sacc, codes_to_f16x2(w0, kSelB01), codes_to_f16x2(w1, kSelB01),
-                      codes_to_f16x2(w0, kSelB23), codes_to_f16x2(w1, kSelB23), qf[s][0],
-                      qf[s][1]);
-      }
-      const int tA = T + 16 * u + g, tB = tA + 8;
-      x[u][0] = tA < t_end ? sacc[0] * ksc[u][0] * sc0 : -INFINITY;
-      x[u][1] = tA < t_end ? sacc[1] * ksc[u][0] * sc1 : -INFINITY;
-      x[u][2] = tB < t_end ? sacc[2] * ksc[u][1] * sc0 : -INFINITY;
-      x[u][3] = tB < t_end ? sacc[3] * ksc[u][1] * sc1 : -INFINITY;
-    }
-    if (has_next) load_k(T + 128);
-
-    // -- online softmax per head (columns 2c, 2c+1); max over the warp's 32 tokens --
-    float mx0 = fmaxf(fmaxf(x[0][0], x[0][2]), fmaxf(x[1][0], x[1][2]));
-    float mx1 = fmaxf(fmaxf(x[0][1], x[0][3]), fmaxf(x[1][1], x[1][3]));
-#pragma unroll
-    for (int o = 4; o < 32; o <<= 1) {
-      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
-      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
-    }
-    if (mx0 > m0 + 8.f) {
-      const float a = ex2(m0 - mx0);
-      m0 = mx0;
-      l0 *= a;
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        oacc[mt][0] *= a;
-        oacc[mt][2] *= a;
-      }
-    }
-    if (mx1 > m1 + 8.f) {
-      const float a = ex2(m1 - mx1);
-      m1 = mx1;
-      l1 *= a;
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        oacc[mt][1] *= a;
-        oacc[mt][3] *= a;
-      }
-    }
-    const float mu0 = (m0 == -INFINITY) ? 0.f : m0;
-    const float mu1 = (m1 == -INFINITY) ? 0.f : m1;
-    uint32_t pb[2][2];  // PV B operand per group: tokens 0-7 and 8-15 of the group
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const float pa0 = ex2(x[u][0] - mu0), pa1 = ex2(x[u][1] - mu1);
-      const float pb0 = ex2(x[u][2] - mu0), pb1 = ex2(x[u][3] - mu1);
-      l0 += pa0 + pb0;
-      l1 += pa1 + pb1;
-      const float wa = vsc[u][0] * pscale, wb = vsc[u][1] * pscale;
-      pb[u][0] = movmatrix_trans(pack_f16x2(pa0 * wa, pa1 * wa));
-      pb[u][1] = movmatrix_trans(pack_f16x2(pb0 * wb, pb1 * wb));
-    }
-
-    // -- O^T += Vcode^T . P'^T --
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      uint32_t r[4][VB / 4];
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4)
-#pragma unroll
-        for (int w = 0; w < VB / 4; ++w) r[q4][w] = vw[u][q4][w] ^ 0x80808080u;
-#pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        const int w = mt >> 1;
-        const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
-        const uint32_t x01 = prmt(r[0][w], r[1][w], sel);  // tokens 2c, 2c+1
-        const uint32_t x89 = prmt(r[2][w], r[3][w], sel);  // tokens 2c+8, 2c+9
-        mma_f16_16816(oacc[mt], codes_to_f16x2(x01, kSelB01), codes_to_f16x2(x01, kSelB23),
-                      codes_to_f16x2(x89, kSelB01), codes_to_f16x2(x89, kSelB23), pb[u][0],
-                      pb[u][1]);
-      }
-    }
-    if (has_next) load_v(T + 128);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_empty(s));
   }
 
-  // ---- merge the 4 warps ----
+  // ---- merge the 4 warps (the stage tiles are free now: every stage has been consumed) ----
+  named_bar_sync(1, 128);
+  float* sm_o = reinterpret_cast<float*>(smem + C::kMergeO);
+  float* sm_m = reinterpret_cast<float*>(smem + C::kMergeM);
+  float* sm_l = reinterpret_cast<float*>(smem + C::kMergeL);
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
     l0 += __shfl_xor_sync(0xffffffffu, l0, o);
     l1 += __shfl_xor_sync(0xffffffffu, l1, o);
   }
   if (g == 0) {
-    sm_m[warp][2 * c] = m0;
-    sm_m[warp][2 * c + 1] = m1;
-    sm_l[warp][2 * c] = l0;
-    sm_l[warp][2 * c + 1] = l1;
+    sm_m[warp * 8 + 2 * c] = m0;
+    sm_m[warp * 8 + 2 * c + 1] = m1;
+    sm_l[warp * 8 + 2 * c] = l0;
+    sm_l[warp * 8 + 2 * c + 1] = l1;
   }
+  const float unscale = (E == kEUnset) ? 0.f : exp2i_or_zero(-E);
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
     const int d0 = VB * g + 2 * mt;
-    sm_o[warp][2 * c][d0] = oacc[mt][0];
-    sm_o[warp][2 * c + 1][d0] = oacc[mt][1];
-    sm_o[warp][2 * c][d0 + 1] = oacc[mt][2];
-    sm_o[warp][2 * c + 1][d0 + 1] = oacc[mt][3];
+    float* ow = sm_o + warp * 8 * D;
+    ow[(2 * c) * D + d0] = oacc[mt][0] * unscale;
+    ow[(2 * c + 1) * D + d0] = oacc[mt][1] * unscale;
+    ow[(2 * c) * D + d0 + 1] = oacc[mt][2] * unscale;
+    ow[(2 * c + 1) * D + d0 + 1] = oacc[mt][3] * unscale;
   }
-  __syncthreads();
+  named_bar_sync(1, 128);
   for (int idx = threadIdx.x; idx < nheads * D; idx += 128) {
     const int h = idx / D, d = idx % D;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, sm_m[w][h]);
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, sm_m[w * 8 + h]);
     float L = 0.f, acc = 0.f;
     if (M != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
-        const float f = (sm_m[w][h] == -INFINITY) ? 0.f : ex2(sm_m[w][h] - M);
-        L += f * sm_l[w][h];
-        acc += f * sm_o[w][h][d];
+        const float mw = sm_m[w * 8 + h];
+        const float f = (mw == -INFINITY) ? 0.f : ex2(mw - M);
+        L += f * sm_l[w * 8 + h];
+        acc += f * sm_o[(w * 8 + h) * D + d];
       }
     }
     const size_t row = (static_cast<size_t>(split) * p.B + b) * p.Hq + head0 + h;
-    p.o_part[row * D + d] = (L > 0.f) ? acc / (L * pscale) : 0.f;
+    p.o_part[row * D + d] = (L > 0.f) ? acc / L : 0.f;
     if (d == 0) p.lse_part[row] = (L > 0.f) ? (M + __log2f(L)) * 0.69314718055994531f : -INFINITY;
   }
 }

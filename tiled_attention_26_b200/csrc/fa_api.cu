@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -54,6 +55,23 @@ int encode_bf16_4d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1,
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+// int8 K or V codes viewed as a 4-D tensor (D, Hkv, keys, B-or-pages); a box is `box_keys`
+// key rows of one KV head.  Rows of 128 bytes are 128B-swizzled in shared memory.
+int encode_u8_4d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1, uint64_t n2,
+                 uint64_t n3, uint32_t box_keys) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return FA_ERR_CUDA;
+  const cuuint64_t dims[4] = {n0, n1, n2, n3};
+  const cuuint64_t strides[3] = {n0, n0 * n1, n0 * n1 * n2};
+  const cuuint32_t box[4] = {static_cast<cuuint32_t>(n0), 1, box_keys, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  n0 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
@@ -156,13 +174,30 @@ fa::DecodeParams decode_params(const void* q, const int8_t* k, const int8_t* v, 
   return p;
 }
 
-// Split kernel over grid (Hkv, splits, B * head blocks), then the merge kernel.
+std::atomic<uint64_t> g_attr_decode[4];
+
+// Split kernel over grid (Hkv, splits, B * head blocks), then the merge kernel.  `keys` is the
+// extent of the key axis of the code tensors (Skv, or the page size), `outer` that of the last
+// axis (B, or the number of pages).
 template <int D, bool kPaged>
-int launch_split_and_combine(const fa::DecodeParams& p, void* o, float* lse, cudaStream_t stream) {
+int launch_split_and_combine(const fa::DecodeParams& p, int keys, int outer, void* o, float* lse,
+                             cudaStream_t stream) {
+  using C = fa::DecodeCfg<D>;
   const long long gz = static_cast<long long>(p.B) * ((p.G + 7) / 8);
   if (p.splits > 65535 || gz > 65535) return FA_ERR_INVALID_ARG;
+  CUtensorMap tk, tv;
+  // a box is one stage (128 keys; past the end of the key axis TMA fills zeros and still counts
+  // the bytes) or, for pages smaller than a stage, one page
+  const uint32_t box = static_cast<uint32_t>(kPaged ? std::min(C::kT, keys) : C::kT);
+  int rc;
+  if ((rc = encode_u8_4d(&tk, p.k, D, p.Hkv, keys, outer, box)) != FA_OK) return rc;
+  if ((rc = encode_u8_4d(&tv, p.v, D, p.Hkv, keys, outer, box)) != FA_OK) return rc;
+  auto kernel = fa::fa_decode_split_kernel<D, kPaged>;
+  if ((rc = ensure_smem_attr(kernel, C::kSmemBytes,
+                             g_attr_decode[(D == 128 ? 2 : 0) + (kPaged ? 1 : 0)])) != FA_OK)
+    return rc;
   dim3 grid(p.Hkv, p.splits, static_cast<unsigned>(gz));
-  fa::fa_decode_split_kernel<D, kPaged><<<grid, 128, 0, stream>>>(p);
+  kernel<<<grid, 160, C::kSmemBytes, stream>>>(tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
   fa::CombineParams cp{};
   cp.o_part = p.o_part;
@@ -195,8 +230,7 @@ int launch_decode(const void* q, const int8_t* k, const int8_t* v, const float* 
                   void* ws, cudaStream_t stream) {
   fa::DecodeParams p = decode_params(q, k, v, ks, vs, B, Hq, Hkv, D, scale, splits, ws);
   p.Skv = Skv;
-  p.chunk = (Skv + splits - 1) / splits;
-  return launch_split_and_combine<D, false>(p, o, lse, stream);
+  return launch_split_and_combine<D, false>(p, Skv, B, o, lse, stream);
 }
 
 template <int D>
@@ -211,7 +245,7 @@ int launch_decode_paged(const void* q, const int8_t* k, const int8_t* v, const f
   p.max_pages = max_pages;
   p.num_pages = num_pages;
   p.page_shift = page_shift;
-  return launch_split_and_combine<D, true>(p, o, lse, stream);
+  return launch_split_and_combine<D, true>(p, 1 << page_shift, num_pages, o, lse, stream);
 }
 
 // Device address of g_noalloc_scratch on the current device.  In host code the symbol name is
