@@ -41,8 +41,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC = {
     # profiles/fa_prefill_kernel_mha_causal.md: 543.66 MB read + 48.50 MB written, one launch
     "prefill": {"24eb617e09b98e34": 592_165_120},
-    # profiles/fa_decode_split_kernel_decode_int8.md: 1107.69 MB read + 3.74 MB written
-    "decode": {"77c2cf5253f1b8fc": 1_111_432_960},
+    # profiles/fa_decode_split_kernel_decode_int8.md: 1,107,554,560 B read + 8,284,160 B written
+    "decode": {"d71c958934a45622": 1_115_838_720},
+    # profiles/fa_decode_split_kernel_decode_int8_paged.md: 424,228,864 B read + 6,737,152 B written
+    "paged_decode": {"d71c958934a45622": 430_966_016},
 }
 
 
@@ -467,7 +469,8 @@ def main():
                 "ms_per_call": pg_ms, "achieved": pg_bytes / (pg_ms * 1e-3) / 1e9,
                 "unit": "GB/s", "peak": peaks["hbm_gbs"],
                 "frac": pg_bytes / (pg_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                "launches": 2 * min(K, 200)},
+                "launches": 2 * min(K, 200),
+                "traffic": NCU_TRAFFIC["paged_decode"].get(source_hash("decode.cuh", "sm100.cuh"))},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 3 * K,
