@@ -39,6 +39,8 @@ def lib():
         L.oracle_decode_int8_rows.argtypes = [_P] * 5 + [_I] * 5 + [_D, _I, _P, _L, _P, _P, _I]
         L.oracle_decode_int8_paged_rows.argtypes = [_P] * 7 + [_I] * 7 + [_D, _I, _P, _L, _P, _P, _I]
         L.oracle_decode_int8_paged_rows.restype = _I
+        L.oracle_unpack_int4.argtypes = [_P, _L, _P]
+        L.oracle_unpack_int4.restype = _I
         for f in (L.oracle_attn_bf16_rows, L.oracle_attn_f64_rows, L.oracle_attn_brute,
                   L.oracle_attn_tiled, L.oracle_decode_int8_rows):
             f.restype = _I
@@ -186,3 +188,30 @@ def decode_int8_paged(q, kp, vp, ksp, vsp, block_table, seqlens, scale, num_spli
     o, lse = decode_int8_paged_rows(q, kp, vp, ksp, vsp, block_table, seqlens, scale, num_splits,
                                     rows, nthreads)
     return o.reshape(B, 1, Hq, D), lse.reshape(B, Hq)
+
+
+def unpack_int4(packed):
+    """Packed INT4 codes (uint8 [..., n]) -> int8 codes [..., 2n]: byte i holds code 2i in its low
+    nibble and code 2i+1 in its high nibble, 4-bit two's complement."""
+    packed = np.ascontiguousarray(packed, dtype=np.uint8)
+    codes = np.empty(packed.shape[:-1] + (2 * packed.shape[-1],), dtype=np.int8)
+    if lib().oracle_unpack_int4(_ptr(packed), packed.size, _ptr(codes)) != 0:
+        raise ValueError("oracle_unpack_int4 rejected its arguments")
+    return codes
+
+
+def decode_int4_rows(q, k4, v4, ks, vs, scale, num_splits, rows, nthreads=0):
+    """Decode over an INT4 KV cache: k4/v4 uint8 [B, Skv, Hkv, D/2] packed codes, ks/vs fp32
+    [B, Hkv, Skv].  The INT8 decode definition over the unpacked codes."""
+    return decode_int8_rows(q, unpack_int4(k4), unpack_int4(v4), ks, vs, scale, num_splits, rows,
+                            nthreads)
+
+
+def decode_int4(q, k4, v4, ks, vs, scale, num_splits=1, nthreads=0):
+    return decode_int8(q, unpack_int4(k4), unpack_int4(v4), ks, vs, scale, num_splits, nthreads)
+
+
+def decode_int4_paged(q, kp4, vp4, ksp, vsp, block_table, seqlens, scale, num_splits=1,
+                      nthreads=0):
+    return decode_int8_paged(q, unpack_int4(kp4), unpack_int4(vp4), ksp, vsp, block_table,
+                             seqlens, scale, num_splits, nthreads)

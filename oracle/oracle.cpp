@@ -32,6 +32,11 @@
 //    dequantised values k_code * k_scale (exact in fp64), one query token per sequence.
 //    With num_splits > 1 it evaluates each key chunk separately and merges the partial
 //    results through their log-sum-exp, the same correction step the online softmax uses.
+//  * INT4 KV cache, the second format of the same KV-compression section ("INT8/INT4").  The
+//    pages give no packing; this project stores two 4-bit two's-complement codes per byte (dim
+//    2i in the low nibble, dim 2i+1 in the high nibble) with one fp32 scale per (token, KV head),
+//    as for INT8.  `oracle_unpack_int4` writes the codes out as int8; the INT4 decode is then
+//    the INT8 decode definition over those codes.
 //  * Dynamic sequence lengths and a paged KV cache -- "Flash Attention on Ascend: three
 //    techniques", version section (sequences of different lengths in one batch) and "Sparse
 //    attention and MLA operators in ops-transformer", section 2.2 (KV cache pages addressed
@@ -458,6 +463,18 @@ int oracle_decode_int8_paged_rows(const uint16_t* q, const int8_t* k, const int8
       }
       lse[r] = L;
     }
+  }
+  return 0;
+}
+
+// Unpack INT4 codes: byte i of `packed` holds code 2i in bits 0-3 and code 2i+1 in bits 4-7,
+// each a 4-bit two's-complement integer in [-8, 7].  Writes 2 * n_bytes int8 codes.
+int oracle_unpack_int4(const uint8_t* packed, int64_t n_bytes, int8_t* codes) {
+  if (n_bytes < 0 || (n_bytes > 0 && (!packed || !codes))) return -1;
+  for (int64_t i = 0; i < n_bytes; ++i) {
+    const int lo = packed[i] & 0xF, hi = (packed[i] >> 4) & 0xF;
+    codes[2 * i] = static_cast<int8_t>(lo >= 8 ? lo - 16 : lo);
+    codes[2 * i + 1] = static_cast<int8_t>(hi >= 8 ? hi - 16 : hi);
   }
   return 0;
 }

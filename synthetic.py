@@ -7,6 +7,8 @@ This module holds no attention arithmetic. It only draws numbers and names workl
   them into two uniforms and then into two N(0,1) values by the Box-Muller transform
   (fp64).  Each value is rounded to fp32 (round-to-nearest-even) and then to bf16
   (round-to-nearest-even).  The result is returned as raw bf16 bit patterns (uint16).
+* ``quantize_int4_per_token`` -- the INT4 recipe: the same with max|x| / 7 and codes in
+  [-7, 7], packed two per byte (dim 2i in the low nibble), 4-bit two's complement.
 * ``quantize_int8_per_token`` -- the INT8 KV-cache recipe of the decode workload:
   symmetric, one fp32 scale per (token, kv-head) equal to max|x| / 127, codes
   ``clamp(rint(x / scale), -127, 127)`` with the division in fp32 and ties to even.
@@ -101,6 +103,23 @@ def quantize_int8_per_token(x_bits: np.ndarray):
     return q, np.ascontiguousarray(np.transpose(sc, (0, 2, 1)))
 
 
+def quantize_int4_per_token(x_bits: np.ndarray):
+    """bf16 bits ``[B, S, H, D]`` -> (packed uint8 ``[B, S, H, D/2]``, fp32 scales ``[B, H, S]``).
+    Symmetric INT4: scale = max|x| / 7 per (token, head), codes clamp(rint(x / scale), -7, 7)
+    (fp32 division, ties to even), two codes per byte: dim 2i in the low nibble, dim 2i+1 in the
+    high nibble, 4-bit two's complement."""
+    x = bf16_bits_to_f32(x_bits)
+    amax = np.max(np.abs(x), axis=-1)
+    sc = (amax / np.float32(7.0)).astype(np.float32)
+    safe = np.where(sc > 0, sc, np.float32(1.0)).astype(np.float32)
+    qf = np.rint((x / safe[..., None]).astype(np.float32))
+    q = np.clip(qf, -7, 7).astype(np.int8)
+    q[sc == 0] = 0
+    nib = (q.astype(np.int16) & 0xF).astype(np.uint8)
+    packed = (nib[..., 0::2] | (nib[..., 1::2] << 4)).astype(np.uint8)
+    return packed, np.ascontiguousarray(np.transpose(sc, (0, 2, 1)))
+
+
 @dataclass(frozen=True)
 class Workload:
     name: str
@@ -145,6 +164,8 @@ WORKLOADS = {
                            note="MQA prefill, Falcon-180B-like head layout"),
     "decode_int8": Workload("decode_int8", 5, 16, 32, 8, 1, 32768, 128, 1, int8_kv=True,
                             num_splits=16, note="GQA decode over an INT8 KV cache"),
+    "decode_int4": Workload("decode_int4", 8, 16, 32, 8, 1, 32768, 128, 1, num_splits=16,
+                            note="GQA decode over an INT4 KV cache (two codes per byte)"),
 }
 
 
@@ -162,6 +183,14 @@ def make_decode_inputs(w: Workload):
     kq, ks = quantize_int8_per_token(k)
     vq, vs = quantize_int8_per_token(v)
     return q, kq, vq, ks, vs
+
+
+def make_decode_int4_inputs(w: Workload):
+    """Q bf16 bits [B,1,Hq,D]; K, V packed INT4 uint8 [B,Skv,Hkv,D/2]; scales fp32 [B,Hkv,Skv]."""
+    q, k, v = make_qkv(w)
+    k4, ks = quantize_int4_per_token(k)
+    v4, vs = quantize_int4_per_token(v)
+    return q, k4, v4, ks, vs
 
 
 # ---------------------------------------------------------------------------------------
@@ -224,10 +253,32 @@ def quantize_int8_per_token_torch(x):
     return q, sc.permute(0, 2, 1).contiguous()
 
 
+def quantize_int4_per_token_torch(x):
+    """torch version of ``quantize_int4_per_token``: bf16 [B,S,H,D] -> (uint8 [B,S,H,D/2],
+    fp32 scales [B,H,S])."""
+    import torch
+    xf = x.to(torch.float32)
+    amax = xf.abs().amax(dim=-1)
+    sc = amax / 7.0
+    safe = torch.where(sc > 0, sc, torch.ones_like(sc))
+    q = torch.clamp(torch.round(xf / safe[..., None]), -7, 7).to(torch.int16)
+    q[sc == 0] = 0
+    nib = (q & 0xF).to(torch.uint8)
+    packed = nib[..., 0::2] | (nib[..., 1::2] << 4)
+    return packed.contiguous(), sc.permute(0, 2, 1).contiguous()
+
+
 def make_qkv_torch(w: Workload, device):
     return (normal_bf16_torch(w.seed(0), w.q_shape(), device),
             normal_bf16_torch(w.seed(1), w.kv_shape(), device),
             normal_bf16_torch(w.seed(2), w.kv_shape(), device))
+
+
+def make_decode_int4_inputs_torch(w: Workload, device):
+    q = normal_bf16_torch(w.seed(0), w.q_shape(), device)
+    k4, ks = quantize_int4_per_token_torch(normal_bf16_torch(w.seed(1), w.kv_shape(), device))
+    v4, vs = quantize_int4_per_token_torch(normal_bf16_torch(w.seed(2), w.kv_shape(), device))
+    return q, k4, v4, ks, vs
 
 
 def make_decode_inputs_torch(w: Workload, device):
