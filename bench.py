@@ -6,8 +6,9 @@ One step = one pass of the whole path over one batch of synthetic input:
     headline metric is quoted on (attention forward TFLOP/s);
   * decode   (fa_decode_int8, split kernel + combine kernel): B=16, Hq=32, Hkv=8, Skv=32768,
     D=128, INT8 KV cache with per-token scales, 16 splits (KV-read GB/s).
-After the timed steps, a short loop of its own times the paged, variable-length decode
-(fa_decode_int8_paged) and reports it under "paged_decode"; it is not part of the step.
+After the timed steps, short loops of their own time the paged, variable-length decode
+(fa_decode_int8_paged, "paged_decode") and the INT4 decode (fa_decode_int4, "int4_decode");
+they are not part of the step.
 Inputs are seeded synthetic N(0,1) draws (see synthetic.py) resident in HBM; both inputs are
 larger than the 126 MB L2 (prefill 268 MB, decode 1.1 GB), so no flush is needed between steps.
 
@@ -122,6 +123,42 @@ def measure_paged_decode(fa, synthetic, torch, dev, stream, steps: int, warmup: 
     if fa.fa_device_status() != 0:
         raise RuntimeError("the paged decode reported a device-side error")
     return a.elapsed_time(b) / steps, paged_decode_bytes(w, sl.cpu().numpy())
+
+
+def int4_decode_bytes(w) -> int:
+    """Algorithmic bytes of one INT4 decode call: packed K and V codes (D/2 bytes per key and
+    head), fp32 scales, bf16 q in and o out, fp32 LSE."""
+    kv = 2 * w.B * w.Skv * w.Hkv * (w.D // 2)
+    scales = 2 * w.B * w.Hkv * w.Skv * 4
+    return kv + scales + 2 * w.B * w.Hq * w.D * 2 + w.B * w.Hq * 4
+
+
+def measure_int4_decode(fa, synthetic, torch, dev, stream, steps: int, warmup: int):
+    """Time fa_decode_int4 on the INT4 workload (its own short loop after the step loop).
+    Returns (ms per call averaged over ``steps`` launches, algorithmic bytes per call)."""
+    w = synthetic.WORKLOADS["decode_int4"]
+    q, k4, v4, ks, vs = synthetic.make_decode_int4_inputs_torch(w, dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(fa.fa_decode_int8_workspace_bytes(w.B, w.Hq, w.D, w.num_splits),
+                     dtype=torch.uint8, device=dev)
+
+    def call():
+        fa.fa_decode_int4(q, k4, v4, ks, vs, num_splits=w.num_splits, scale=w.scale, o=o,
+                          lse=lse, workspace=ws, stream=stream)
+
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        call()
+    b.record(stream)
+    torch.cuda.synchronize()
+    if fa.fa_device_status() != 0:
+        raise RuntimeError("the INT4 decode reported a device-side error")
+    return a.elapsed_time(b) / steps, int4_decode_bytes(w)
 
 
 class ClockSampler:
@@ -376,6 +413,9 @@ def main():
     pg_ms, pg_bytes = measure_paged_decode(fa, synthetic, torch, dev, stream,
                                            steps=min(K, 200), warmup=max(3, args.warmup // 4))
     pg_ms = max_over_ranks(pg_ms)
+    i4_ms, i4_bytes = measure_int4_decode(fa, synthetic, torch, dev, stream,
+                                          steps=min(K, 200), warmup=max(3, args.warmup // 4))
+    i4_ms = max_over_ranks(i4_ms)
 
     # ---- end to end through the public API, host buffers, copies inside the timed region ----
     e2e = None
@@ -471,6 +511,14 @@ def main():
                 "frac": pg_bytes / (pg_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                 "launches": 2 * min(K, 200),
                 "traffic": NCU_TRAFFIC["paged_decode"].get(source_hash("decode.cuh", "sm100.cuh"))},
+            "int4_decode": {
+                "workload": "decode_int4: B=16, Hq=32, Hkv=8, Skv=32768, D=128, INT4 KV (two codes "
+                            f"per byte, per-token scales, {i4_bytes / 1e6:.1f} MB per call), 16 splits",
+                "kernel": "fa_decode_split_kernel<128, contiguous, 4-bit> + fa_decode_combine_kernel<128>",
+                "ms_per_call": i4_ms, "achieved": i4_bytes / (i4_ms * 1e-3) / 1e9,
+                "unit": "GB/s", "peak": peaks["hbm_gbs"],
+                "frac": i4_bytes / (i4_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                "launches": 2 * min(K, 200)},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 3 * K,

@@ -182,6 +182,33 @@ FA_API int fa_decode_int8_paged(const void* q, const int8_t* k_pages, const int8
                                 int num_splits, void* workspace, size_t workspace_bytes,
                                 void* stream);
 
+/*
+ * Decode step over an INT4 KV cache (the KV-compression section of "Flash Attention on Ascend:
+ * three techniques" names INT4 beside INT8; the pages give no packing, this library's format
+ * is the following).  Two codes per byte: byte i of a key row holds dim 2i in bits 0-3 and dim
+ * 2i+1 in bits 4-7, each a 4-bit two's-complement code; element value = code * scale of its
+ * (token, KV head).
+ *   k, v    uint8 [B, Skv, Hkv, D/2]   packed codes
+ *   every other argument, layout, status code and the split semantics are those of
+ *   fa_decode_int8 (the workspace size is fa_decode_int8_workspace_bytes).
+ */
+FA_API int fa_decode_int4(const void* q, const uint8_t* k, const uint8_t* v, const float* k_scale,
+                          const float* v_scale, void* o, float* lse, int B, int Hq, int Hkv,
+                          int Skv, int D, float scale, int num_splits, void* workspace,
+                          size_t workspace_bytes, void* stream);
+
+/*
+ * Paged, variable-length decode over an INT4 KV cache: fa_decode_int8_paged with
+ * k_pages, v_pages uint8 [num_pages, page_size, Hkv, D/2] packed as for fa_decode_int4.
+ */
+FA_API int fa_decode_int4_paged(const void* q, const uint8_t* k_pages, const uint8_t* v_pages,
+                                const float* k_scale_pages, const float* v_scale_pages,
+                                const int32_t* block_table, const int32_t* seqlens, void* o,
+                                float* lse, int B, int Hq, int Hkv, int page_size,
+                                int max_pages_per_seq, int num_pages, int D, float scale,
+                                int num_splits, void* workspace, size_t workspace_bytes,
+                                void* stream);
+
 /* Static, human-readable name of a status code.  Never NULL. */
 FA_API const char* fa_status_string(int status);
 

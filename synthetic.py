@@ -368,23 +368,26 @@ def paged_layout(w: PagedDecodeWorkload, seqlens=None):
     return seqlens.astype(np.int32), bt, num_pages
 
 
-def make_paged_decode_inputs(w: PagedDecodeWorkload, seqlens=None):
-    """q bf16 bits [B,1,Hq,D]; K/V int8 pages, fp32 scale pages, block_table, seqlens."""
+def make_paged_decode_inputs(w: PagedDecodeWorkload, seqlens=None, bits: int = 8):
+    """q bf16 bits [B,1,Hq,D]; K/V code pages (int8, or packed INT4 uint8 with ``bits=4``),
+    fp32 scale pages, block_table, seqlens."""
     sl, bt, num_pages = paged_layout(w, seqlens)
     q = normal_bf16(w.seed(0), (w.B, 1, w.Hq, w.D))
     shape = (num_pages, w.page_size, w.Hkv, w.D)
-    kp, ksp = quantize_int8_per_token(normal_bf16(w.seed(1), shape))
-    vp, vsp = quantize_int8_per_token(normal_bf16(w.seed(2), shape))
+    quant = quantize_int8_per_token if bits == 8 else quantize_int4_per_token
+    kp, ksp = quant(normal_bf16(w.seed(1), shape))
+    vp, vsp = quant(normal_bf16(w.seed(2), shape))
     return q, kp, vp, ksp, vsp, bt, sl
 
 
-def make_paged_decode_inputs_torch(w: PagedDecodeWorkload, device, seqlens=None):
+def make_paged_decode_inputs_torch(w: PagedDecodeWorkload, device, seqlens=None, bits: int = 8):
     """The same inputs drawn with the torch generator on ``device`` (large workloads)."""
     import torch
     sl, bt, num_pages = paged_layout(w, seqlens)
     q = normal_bf16_torch(w.seed(0), (w.B, 1, w.Hq, w.D), device)
     shape = (num_pages, w.page_size, w.Hkv, w.D)
-    kp, ksp = quantize_int8_per_token_torch(normal_bf16_torch(w.seed(1), shape, device))
-    vp, vsp = quantize_int8_per_token_torch(normal_bf16_torch(w.seed(2), shape, device))
+    quant = quantize_int8_per_token_torch if bits == 8 else quantize_int4_per_token_torch
+    kp, ksp = quant(normal_bf16_torch(w.seed(1), shape, device))
+    vp, vsp = quant(normal_bf16_torch(w.seed(2), shape, device))
     return (q, kp, vp, ksp, vsp, torch.from_numpy(bt).to(device),
             torch.from_numpy(sl).to(device))

@@ -32,7 +32,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("fa_fwd", "fa_decode_int8", "fa_decode_int8_workspace_bytes", "fa_status_string",
               "fa_device_status", "fa_selftest_bounded_wait", "fa_decode_int8_noalloc",
-              "fa_decode_int8_paged"):
+              "fa_decode_int8_paged", "fa_decode_int4", "fa_decode_int4_paged"):
         assert n in names
 
 
@@ -133,6 +133,26 @@ def paged(L, q=FAKE, k=FAKE, v=FAKE, ks=FAKE, vs=FAKE, bt=FAKE, sl=FAKE, o=FAKE,
 ])
 def test_paged_decode_rejects(L, kw, code):
     assert paged(L, **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(k=None), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(Skv=0), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(D=96), fa.STATUS["FA_ERR_UNSUPPORTED"]),
+    (dict(v=FAKE + 4), fa.STATUS["FA_ERR_ALIGNMENT"]),
+    (dict(ws_bytes=16), fa.STATUS["FA_ERR_WORKSPACE"]),
+])
+def test_int4_decode_rejects(L, kw, code):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, ks=FAKE, vs=FAKE, o=FAKE, lse=None, B=2, Hq=8, Hkv=2,
+                Skv=100, D=128, scale=0.1, splits=4, ws=FAKE, ws_bytes=None)
+    args.update(kw)
+    if args["ws_bytes"] is None:
+        args["ws_bytes"] = L.fa_decode_int8_workspace_bytes(args["B"], args["Hq"], args["D"],
+                                                            args["splits"])
+    a = args
+    assert L.fa_decode_int4(a["q"], a["k"], a["v"], a["ks"], a["vs"], a["o"], a["lse"], a["B"],
+                            a["Hq"], a["Hkv"], a["Skv"], a["D"], a["scale"], a["splits"], a["ws"],
+                            a["ws_bytes"], None) == code
 
 
 def test_workspace_bytes(L):

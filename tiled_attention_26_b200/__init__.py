@@ -13,8 +13,9 @@ import math
 import os
 
 __all__ = ["FaError", "lib", "fa_fwd", "fa_decode_int8", "fa_decode_int8_paged",
-           "fa_decode_int8_workspace_bytes", "fa_status_string", "fa_device_status",
-           "fa_selftest_bounded_wait", "LIB_PATH", "STATUS"]
+           "fa_decode_int4", "fa_decode_int4_paged", "fa_decode_int8_workspace_bytes",
+           "fa_status_string", "fa_device_status", "fa_selftest_bounded_wait", "LIB_PATH",
+           "STATUS"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
 
@@ -59,6 +60,10 @@ def lib() -> ctypes.CDLL:
         L.fa_decode_int8.restype = _I
         L.fa_decode_int8_paged.argtypes = [_P] * 9 + [_I] * 7 + [_F, _I, _P, _Z, _P]
         L.fa_decode_int8_paged.restype = _I
+        L.fa_decode_int4.argtypes = [_P] * 7 + [_I] * 5 + [_F, _I, _P, _Z, _P]
+        L.fa_decode_int4.restype = _I
+        L.fa_decode_int4_paged.argtypes = [_P] * 9 + [_I] * 7 + [_F, _I, _P, _Z, _P]
+        L.fa_decode_int4_paged.restype = _I
         L.fa_status_string.argtypes = [_I]
         L.fa_status_string.restype = ctypes.c_char_p
         L.fa_device_status.argtypes = [_P]
@@ -130,20 +135,20 @@ def fa_decode_int8_workspace_bytes(B: int, Hq: int, D: int, num_splits: int) -> 
     return int(lib().fa_decode_int8_workspace_bytes(int(B), int(Hq), int(D), int(num_splits)))
 
 
-def fa_decode_int8(q, k, v, k_scale, v_scale, num_splits: int = 16, scale: float | None = None,
-                   o=None, lse=None, workspace=None, return_lse: bool = True, stream=None):
-    """Decode step over an INT8 KV cache.  q: bf16 [B, 1, Hq, D]; k, v: int8 [B, Skv, Hkv, D];
-    k_scale, v_scale: fp32 [B, Hkv, Skv].  Returns ``(o, lse)`` with o bf16 [B, 1, Hq, D] and
-    lse fp32 [B, Hq]."""
+def _decode(bits, q, k, v, k_scale, v_scale, num_splits, scale, o, lse, workspace, return_lse,
+            stream):
     import torch
+    name = f"fa_decode_int{bits}"
     B, one, Hq, D = q.shape
     if one != 1:
         raise ValueError("decode takes one query token per sequence")
     Skv, Hkv = k.shape[1], k.shape[2]
     dev = q.device
+    code = torch.int8 if bits == 8 else torch.uint8
+    row = D if bits == 8 else D // 2
     _check(q, "q", torch.bfloat16, (B, 1, Hq, D), dev)
-    _check(k, "k", torch.int8, (B, Skv, Hkv, D), dev)
-    _check(v, "v", torch.int8, (B, Skv, Hkv, D), dev)
+    _check(k, "k", code, (B, Skv, Hkv, row), dev)
+    _check(v, "v", code, (B, Skv, Hkv, row), dev)
     _check(k_scale, "k_scale", torch.float32, (B, Hkv, Skv), dev)
     _check(v_scale, "v_scale", torch.float32, (B, Hkv, Skv), dev)
     if o is None:
@@ -158,35 +163,50 @@ def fa_decode_int8(q, k, v, k_scale, v_scale, num_splits: int = 16, scale: float
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    rc = lib().fa_decode_int8(q.data_ptr(), k.data_ptr(), v.data_ptr(), k_scale.data_ptr(),
+    rc = getattr(lib(), name)(q.data_ptr(), k.data_ptr(), v.data_ptr(), k_scale.data_ptr(),
                               v_scale.data_ptr(), o.data_ptr(),
                               lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Skv, D,
                               float(scale), int(num_splits), workspace.data_ptr(),
                               workspace.numel() * workspace.element_size(), _stream_ptr(stream))
     if rc != 0:
-        raise FaError(rc, "fa_decode_int8")
+        raise FaError(rc, name)
     return o, lse
 
 
-def fa_decode_int8_paged(q, k_pages, v_pages, k_scale_pages, v_scale_pages, block_table,
-                         seqlens, num_splits: int = 16, scale: float | None = None, o=None,
-                         lse=None, workspace=None, return_lse: bool = True, stream=None):
-    """Decode step over a paged INT8 KV cache with one length per sequence.
-    q: bf16 [B, 1, Hq, D]; k_pages, v_pages: int8 [num_pages, P, Hkv, D]; k_scale_pages,
-    v_scale_pages: fp32 [num_pages, Hkv, P]; block_table: int32 [B, max_pages]; seqlens: int32
-    [B] (both on the device).  Returns ``(o, lse)`` with o bf16 [B, 1, Hq, D], lse fp32 [B, Hq]."""
+def fa_decode_int8(q, k, v, k_scale, v_scale, num_splits: int = 16, scale: float | None = None,
+                   o=None, lse=None, workspace=None, return_lse: bool = True, stream=None):
+    """Decode step over an INT8 KV cache.  q: bf16 [B, 1, Hq, D]; k, v: int8 [B, Skv, Hkv, D];
+    k_scale, v_scale: fp32 [B, Hkv, Skv].  Returns ``(o, lse)`` with o bf16 [B, 1, Hq, D] and
+    lse fp32 [B, Hq]."""
+    return _decode(8, q, k, v, k_scale, v_scale, num_splits, scale, o, lse, workspace,
+                   return_lse, stream)
+
+
+def fa_decode_int4(q, k, v, k_scale, v_scale, num_splits: int = 16, scale: float | None = None,
+                   o=None, lse=None, workspace=None, return_lse: bool = True, stream=None):
+    """Decode step over an INT4 KV cache.  k, v: uint8 [B, Skv, Hkv, D/2], two 4-bit
+    two's-complement codes per byte (dim 2i in the low nibble); otherwise as fa_decode_int8."""
+    return _decode(4, q, k, v, k_scale, v_scale, num_splits, scale, o, lse, workspace,
+                   return_lse, stream)
+
+
+def _decode_paged(bits, q, k_pages, v_pages, k_scale_pages, v_scale_pages, block_table, seqlens,
+                  num_splits, scale, o, lse, workspace, return_lse, stream):
     import torch
+    name = f"fa_decode_int{bits}_paged"
     B, one, Hq, D = q.shape
     if one != 1:
         raise ValueError("decode takes one query token per sequence")
     if k_pages.dim() != 4 or block_table.dim() != 2:
-        raise ValueError("k_pages must be [num_pages, P, Hkv, D], block_table [B, max_pages]")
+        raise ValueError("k_pages must be [num_pages, P, Hkv, row], block_table [B, max_pages]")
     num_pages, P, Hkv = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
     max_pages = block_table.shape[1]
     dev = q.device
+    code = torch.int8 if bits == 8 else torch.uint8
+    row = D if bits == 8 else D // 2
     _check(q, "q", torch.bfloat16, (B, 1, Hq, D), dev)
-    _check(k_pages, "k_pages", torch.int8, (num_pages, P, Hkv, D), dev)
-    _check(v_pages, "v_pages", torch.int8, (num_pages, P, Hkv, D), dev)
+    _check(k_pages, "k_pages", code, (num_pages, P, Hkv, row), dev)
+    _check(v_pages, "v_pages", code, (num_pages, P, Hkv, row), dev)
     _check(k_scale_pages, "k_scale_pages", torch.float32, (num_pages, Hkv, P), dev)
     _check(v_scale_pages, "v_scale_pages", torch.float32, (num_pages, Hkv, P), dev)
     _check(block_table, "block_table", torch.int32, (B, max_pages), dev)
@@ -203,15 +223,35 @@ def fa_decode_int8_paged(q, k_pages, v_pages, k_scale_pages, v_scale_pages, bloc
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    rc = lib().fa_decode_int8_paged(
+    rc = getattr(lib(), name)(
         q.data_ptr(), k_pages.data_ptr(), v_pages.data_ptr(), k_scale_pages.data_ptr(),
         v_scale_pages.data_ptr(), block_table.data_ptr(), seqlens.data_ptr(), o.data_ptr(),
         lse.data_ptr() if lse is not None else None, B, Hq, Hkv, P, max_pages, num_pages, D,
         float(scale), int(num_splits), workspace.data_ptr(),
         workspace.numel() * workspace.element_size(), _stream_ptr(stream))
     if rc != 0:
-        raise FaError(rc, "fa_decode_int8_paged")
+        raise FaError(rc, name)
     return o, lse
+
+
+def fa_decode_int8_paged(q, k_pages, v_pages, k_scale_pages, v_scale_pages, block_table,
+                         seqlens, num_splits: int = 16, scale: float | None = None, o=None,
+                         lse=None, workspace=None, return_lse: bool = True, stream=None):
+    """Decode step over a paged INT8 KV cache with one length per sequence.
+    q: bf16 [B, 1, Hq, D]; k_pages, v_pages: int8 [num_pages, P, Hkv, D]; k_scale_pages,
+    v_scale_pages: fp32 [num_pages, Hkv, P]; block_table: int32 [B, max_pages]; seqlens: int32
+    [B] (both on the device).  Returns ``(o, lse)`` with o bf16 [B, 1, Hq, D], lse fp32 [B, Hq]."""
+    return _decode_paged(8, q, k_pages, v_pages, k_scale_pages, v_scale_pages, block_table,
+                         seqlens, num_splits, scale, o, lse, workspace, return_lse, stream)
+
+
+def fa_decode_int4_paged(q, k_pages, v_pages, k_scale_pages, v_scale_pages, block_table,
+                         seqlens, num_splits: int = 16, scale: float | None = None, o=None,
+                         lse=None, workspace=None, return_lse: bool = True, stream=None):
+    """Paged, variable-length decode over an INT4 KV cache: k_pages, v_pages uint8
+    [num_pages, P, Hkv, D/2] packed as for fa_decode_int4; otherwise as fa_decode_int8_paged."""
+    return _decode_paged(4, q, k_pages, v_pages, k_scale_pages, v_scale_pages, block_table,
+                         seqlens, num_splits, scale, o, lse, workspace, return_lse, stream)
 
 
 def fa_device_status(stream=None) -> int:

@@ -130,6 +130,12 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
   return r;
 }
 
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+  uint32_t r;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(addr));
+  return r;
+}
+
 __device__ __forceinline__ float lds32f(uint32_t addr) {
   float r;
   asm volatile("ld.shared.f32 %0, [%1];" : "=f"(r) : "r"(addr));
@@ -158,13 +164,14 @@ __device__ __forceinline__ void cp_async_wait_all() {
 #endif
 
 // Shared-memory plan of the split kernel.  A stage holds 128 keys: the K and V code tiles
-// ([128 rows][D bytes], 128B-swizzled for D = 128 so that the row-per-lane fragment reads are
-// conflict free) and their fp32 scales.
-template <int D>
+// ([128 rows][kRow bytes], swizzled like the TMA box so that the row-per-lane fragment reads
+// spread over the banks) and their fp32 scales.
+template <int D, int kBits>
 struct DecodeCfg {
   static constexpr int kT = 128;                  // keys per stage
   static constexpr int kStages = FA_DECODE_STAGES;
-  static constexpr int kTile = kT * D;            // bytes of one K or V code tile
+  static constexpr int kRow = D * kBits / 8;      // bytes of one key row of codes
+  static constexpr int kTile = kT * kRow;         // bytes of one K or V code tile
   static constexpr int kStageBytes = 2 * kTile;
   static constexpr int kScaleOff = kStages * kStageBytes;  // fp32 [stages][K, V][kT]
   static constexpr int kBarOff = kScaleOff + kStages * 2 * kT * 4;
@@ -173,7 +180,6 @@ struct DecodeCfg {
   static constexpr int kPageOff = kMiscOff + 16;
   static constexpr int kEnd = kPageOff + 4 * kPageStage;
   static constexpr int kSmemBytes = kEnd + 1024;           // + alignment of the dynamic base
-  static constexpr bool kSwizzle = (D == 128);
   // merge buffers, reused from the stage tiles once the key loop is over
   static constexpr int kMergeO = 0;                        // fp32 [4 warps][8 heads][D]
   static constexpr int kMergeM = 4 * 8 * D * 4;            // fp32 [4][8]
@@ -181,22 +187,38 @@ struct DecodeCfg {
   static_assert(kMergeL + 4 * 8 * 4 <= kScaleOff, "merge buffers must fit in the stage tiles");
 };
 
-// Byte offset of 16-byte chunk `chunk` of row `row` in a code tile whose base is 1024-aligned.
-template <int D>
-__device__ __forceinline__ uint32_t tile_off(int row, int chunk) {
-  if constexpr (D == 128) return row * 128 + ((chunk ^ (row & 7)) << 4);
-  else return row * D + (chunk << 4);
+// Byte offset in a code tile (base aligned to 1024 bytes) of byte `off` of the unswizzled tile:
+// rows of 128 / 64 bytes use the TMA 128B / 64B swizzle (16-byte chunk index XOR address bits
+// 7..9 / 7..8); 32-byte rows are stored plainly.
+template <int kRow>
+__device__ __forceinline__ uint32_t swz(uint32_t off) {
+  if constexpr (kRow == 128) return off ^ (((off >> 7) & 7u) << 4);
+  else if constexpr (kRow == 64) return off ^ (((off >> 7) & 3u) << 4);
+  else return off;
 }
 
-template <int D, bool kPaged>
+// INT4: nibbles at bits [s, s+4) and [s+16, s+20) of an offset-binary word (code + 8) -> fp16x2
+// {code_lo, code_hi} exactly: 1024 + n in fp16 has unit mantissa steps, minus 1032 leaves n - 8.
+__device__ __forceinline__ uint32_t nibbles_to_f16x2(uint32_t biased, int s) {
+  const uint32_t h = ((biased >> s) & 0x000F000Fu) | 0x64006400u;
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(h), "r"(0x64086408u));
+  return d;
+}
+
+template <int D, bool kPaged, int kBits>
 __global__ void __launch_bounds__(160, 1) fa_decode_split_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const DecodeParams p) {
-  using C = DecodeCfg<D>;
-  constexpr int KS = D / 16;  // QK k-steps
-  constexpr int MT = D / 16;  // PV m-tiles (16 output dims each)
-  constexpr int VB = D / 8;   // V bytes per thread per key
-  constexpr int QB = D / 4;   // K bytes per thread per key (its share of the dims)
+  using C = DecodeCfg<D, kBits>;
+  constexpr int KS = D / 16;            // QK k-steps
+  constexpr int MT = D / 16;            // PV m-tiles (16 output dims each)
+  constexpr int QD = D / 4;             // QK: dims of each key row held by one thread
+  constexpr int QW = QD * kBits / 32;   // ... as 32-bit words
+  constexpr int DPT = D / 8;            // PV: output dims of one thread
+  constexpr int VB = DPT * kBits / 8;   // ... as bytes of each V row
+  constexpr int VW = (VB + 3) / 4;      // ... as 32-bit words
+  constexpr uint32_t kBias = kBits == 8 ? 0x80808080u : 0x88888888u;  // to offset binary
   // the merge kernel may be scheduled as soon as every CTA of this grid has started
   asm volatile("griddepcontrol.launch_dependents;");
 
@@ -305,7 +327,7 @@ __global__ void __launch_bounds__(160, 1) fa_decode_split_kernel(
         mbar_arrive_expect_tx(bar_full(s), C::kStageBytes);
         const uint32_t kt = sb + s * C::kStageBytes, vt = kt + C::kTile;
         for (int t = t0; t < t0 + C::kT; t += box_t) {
-          const uint32_t off = (t - t0) * D;
+          const uint32_t off = (t - t0) * C::kRow;  // box_t divides kT: stays inside the tile
           if constexpr (kPaged) {
             // a box past the split's last key reads the split's last page (its keys are masked)
             const int pg = page_of(min(t, t_end - 1));
@@ -338,8 +360,9 @@ __global__ void __launch_bounds__(160, 1) fa_decode_split_kernel(
   const int g = lane >> 2, c = lane & 3;
 
   // ---- Q as the B operand of the QK mma, fp16, scaled by 2^eq per head (exact) ----
-  // Thread c holds dims [QB*c, QB*c + QB) of its head: k-step s, element e is dim QB*c + 4s + e,
-  // the same dims its K fragment reads from each key row.
+  // Thread c holds dims [QD*c, QD*c + QD) of its head, in the order its K fragment takes them
+  // from each key row: INT8 k-step s, element e is dim 4s + e of the block; INT4 k-step 2j + h
+  // takes nibbles (2h, 2h+4) and (2h+1, 2h+5) of word j, i.e. dims 8j + 2h + {0, 4, 1, 5}.
   uint32_t qf[KS][2];
   float sc_mine;
   {
@@ -351,7 +374,8 @@ __global__ void __launch_bounds__(160, 1) fa_decode_split_kernel(
     for (int s = 0; s < KS; ++s)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        qv[s][e] = hv ? bf16_bits_to_float(qrow[QB * c + 4 * s + e]) : 0.f;
+        const int dim = kBits == 8 ? 4 * s + e : 8 * (s >> 1) + 2 * (s & 1) + (e >> 1) + 4 * (e & 1);
+        qv[s][e] = hv ? bf16_bits_to_float(qrow[QD * c + dim]) : 0.f;
         amax = fmaxf(amax, fabsf(qv[s][e]));
       }
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
@@ -391,27 +415,40 @@ __global__ void __launch_bounds__(160, 1) fa_decode_split_kernel(
       float x[2][4];
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        uint32_t kw[2][KS];
+        uint32_t kw[2][QW];  // this thread's words of rows g and g + 8 of the group
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
-          const int row = r_w + 16 * u + g + 8 * rr;
-          if constexpr (D == 128) {
-            const uint4 lo = lds128(kt + tile_off<D>(row, 2 * c));
-            const uint4 hi = lds128(kt + tile_off<D>(row, 2 * c + 1));
-            kw[rr][0] = lo.x; kw[rr][1] = lo.y; kw[rr][2] = lo.z; kw[rr][3] = lo.w;
-            kw[rr][4 % KS] = hi.x; kw[rr][5 % KS] = hi.y; kw[rr][6 % KS] = hi.z; kw[rr][7 % KS] = hi.w;
-          } else {
-            const uint4 lo = lds128(kt + tile_off<D>(row, c));
-            kw[rr][0] = lo.x; kw[rr][1] = lo.y; kw[rr][2 % KS] = lo.z; kw[rr][3 % KS] = lo.w;
+          const uint32_t row0 = (r_w + 16 * u + g + 8 * rr) * C::kRow + QD * kBits / 8 * c;
+#pragma unroll
+          for (int w4 = 0; w4 < QW; w4 += 4) {
+            if constexpr (QW >= 4) {
+              const uint4 x = lds128(kt + swz<C::kRow>(row0 + 4 * w4));
+              kw[rr][w4] = x.x ^ kBias;
+              kw[rr][(w4 + 1) % QW] = x.y ^ kBias;
+              kw[rr][(w4 + 2) % QW] = x.z ^ kBias;
+              kw[rr][(w4 + 3) % QW] = x.w ^ kBias;
+            } else {
+              const uint2 x = lds64(kt + swz<C::kRow>(row0));
+              kw[rr][0] = x.x ^ kBias;
+              kw[rr][1 % QW] = x.y ^ kBias;
+            }
           }
         }
         float sacc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int st = 0; st < KS; ++st) {
-          const uint32_t w0 = kw[0][st] ^ 0x80808080u, w1 = kw[1][st] ^ 0x80808080u;
-          mma_f16_16816(sacc, codes_to_f16x2(w0, kSelB01), codes_to_f16x2(w1, kSelB01),
-                        codes_to_f16x2(w0, kSelB23), codes_to_f16x2(w1, kSelB23), qf[st][0],
-                        qf[st][1]);
+          if constexpr (kBits == 8) {
+            const uint32_t w0 = kw[0][st], w1 = kw[1][st];
+            mma_f16_16816(sacc, codes_to_f16x2(w0, kSelB01), codes_to_f16x2(w1, kSelB01),
+                          codes_to_f16x2(w0, kSelB23), codes_to_f16x2(w1, kSelB23), qf[st][0],
+                          qf[st][1]);
+          } else {
+            const uint32_t w0 = kw[0][st >> 1], w1 = kw[1][st >> 1];
+            const int sh = 8 * (st & 1);
+            mma_f16_16816(sacc, nibbles_to_f16x2(w0, sh), nibbles_to_f16x2(w1, sh),
+                          nibbles_to_f16x2(w0, sh + 4), nibbles_to_f16x2(w1, sh + 4), qf[st][0],
+                          qf[st][1]);
+          }
         }
         const int rA = r_w + 16 * u + g, rB = rA + 8;
         const int tA = T + 16 * u + g, tB = tA + 8;
@@ -497,31 +534,51 @@ __global__ void __launch_bounds__(160, 1) fa_decode_split_kernel(
       // -- O^T += Vcode^T . P'^T --
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
-        uint32_t r[4][VB / 4];
+        uint32_t r[4][VW];  // this thread's words of keys 2c, 2c+1, 2c+8, 2c+9 of the group
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           const int row = r_w + 16 * u + 2 * c + (q4 & 1) + 8 * (q4 >> 1);
+          const uint32_t off = swz<C::kRow>(row * C::kRow + VB * g);
           if constexpr (VB == 16) {
-            const uint4 v4 = lds128(vt + tile_off<D>(row, g));
-            r[q4][0] = v4.x ^ 0x80808080u;
-            r[q4][1 % (VB / 4)] = v4.y ^ 0x80808080u;
-            r[q4][2 % (VB / 4)] = v4.z ^ 0x80808080u;
-            r[q4][3 % (VB / 4)] = v4.w ^ 0x80808080u;
+            const uint4 x = lds128(vt + off);
+            r[q4][0] = x.x ^ kBias;
+            r[q4][1 % VW] = x.y ^ kBias;
+            r[q4][2 % VW] = x.z ^ kBias;
+            r[q4][3 % VW] = x.w ^ kBias;
+          } else if constexpr (VB == 8) {
+            const uint2 x = lds64(vt + off);
+            r[q4][0] = x.x ^ kBias;
+            r[q4][1 % VW] = x.y ^ kBias;
           } else {
-            const uint2 v2 = lds64(vt + row * D + VB * g);
-            r[q4][0] = v2.x ^ 0x80808080u;
-            r[q4][1 % (VB / 4)] = v2.y ^ 0x80808080u;
+            r[q4][0] = lds32(vt + off) ^ kBias;
           }
         }
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
-          const int w = mt >> 1;
-          const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
-          const uint32_t x01 = prmt(r[0][w], r[1][w], sel);  // keys 2c, 2c+1
-          const uint32_t x89 = prmt(r[2][w], r[3][w], sel);  // keys 2c+8, 2c+9
-          mma_f16_16816(oacc[mt], codes_to_f16x2(x01, kSelB01), codes_to_f16x2(x01, kSelB23),
-                        codes_to_f16x2(x89, kSelB01), codes_to_f16x2(x89, kSelB23), pb[u][0],
-                        pb[u][1]);
+          // output dims 2mt and 2mt+1 of this thread's block: INT8 bytes 2mt, 2mt+1; INT4 the
+          // two nibbles of byte mt
+          uint32_t a0, a1, a2, a3;
+          if constexpr (kBits == 8) {
+            const int w = mt >> 1;
+            const uint32_t sel = (mt & 1) ? 0x7362u : 0x5140u;
+            const uint32_t x01 = prmt(r[0][w], r[1][w], sel);  // keys 2c, 2c+1
+            const uint32_t x89 = prmt(r[2][w], r[3][w], sel);  // keys 2c+8, 2c+9
+            a0 = codes_to_f16x2(x01, kSelB01);
+            a1 = codes_to_f16x2(x01, kSelB23);
+            a2 = codes_to_f16x2(x89, kSelB01);
+            a3 = codes_to_f16x2(x89, kSelB23);
+          } else {
+            const int w = mt >> 2;
+            const uint32_t sel = (mt & 2) ? 0x7632u : 0x5410u;
+            const uint32_t x01 = prmt(r[0][w], r[1][w], sel);  // [k0.b, k0.b', k1.b, k1.b']
+            const uint32_t x89 = prmt(r[2][w], r[3][w], sel);
+            const int sh = 8 * (mt & 1);
+            a0 = nibbles_to_f16x2(x01, sh);
+            a1 = nibbles_to_f16x2(x01, sh + 4);
+            a2 = nibbles_to_f16x2(x89, sh);
+            a3 = nibbles_to_f16x2(x89, sh + 4);
+          }
+          mma_f16_16816(oacc[mt], a0, a1, a2, a3, pb[u][0], pb[u][1]);
         }
       }
     }
@@ -548,7 +605,7 @@ __global__ void __launch_bounds__(160, 1) fa_decode_split_kernel(
   const float unscale = (E == kEUnset) ? 0.f : exp2i_or_zero(-E);
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
-    const int d0 = VB * g + 2 * mt;
+    const int d0 = DPT * g + 2 * mt;
     float* ow = sm_o + warp * 8 * D;
     ow[(2 * c) * D + d0] = oacc[mt][0] * unscale;
     ow[(2 * c + 1) * D + d0] = oacc[mt][1] * unscale;

@@ -59,8 +59,9 @@ int encode_bf16_4d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1,
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
-// int8 K or V codes viewed as a 4-D tensor (D, Hkv, keys, B-or-pages); a box is `box_keys`
-// key rows of one KV head.  Rows of 128 bytes are 128B-swizzled in shared memory.
+// K or V codes viewed as a 4-D byte tensor (row bytes, Hkv, keys, B-or-pages); a box is
+// `box_keys` key rows of one KV head.  Rows of 128 / 64 bytes are 128B / 64B-swizzled in shared
+// memory, 32-byte rows are stored plainly.
 int encode_u8_4d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1, uint64_t n2,
                  uint64_t n3, uint32_t box_keys) {
   EncodeTiledFn fn = encode_fn();
@@ -71,7 +72,9 @@ int encode_u8_4d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1, u
   const cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  n0 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  n0 == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                  : n0 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                             : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
@@ -174,15 +177,15 @@ fa::DecodeParams decode_params(const void* q, const int8_t* k, const int8_t* v, 
   return p;
 }
 
-std::atomic<uint64_t> g_attr_decode[4];
+std::atomic<uint64_t> g_attr_decode[8];
 
 // Split kernel over grid (Hkv, splits, B * head blocks), then the merge kernel.  `keys` is the
 // extent of the key axis of the code tensors (Skv, or the page size), `outer` that of the last
 // axis (B, or the number of pages).
-template <int D, bool kPaged>
+template <int D, bool kPaged, int kBits>
 int launch_split_and_combine(const fa::DecodeParams& p, int keys, int outer, void* o, float* lse,
                              cudaStream_t stream) {
-  using C = fa::DecodeCfg<D>;
+  using C = fa::DecodeCfg<D, kBits>;
   const long long gz = static_cast<long long>(p.B) * ((p.G + 7) / 8);
   if (p.splits > 65535 || gz > 65535) return FA_ERR_INVALID_ARG;
   CUtensorMap tk, tv;
@@ -190,12 +193,11 @@ int launch_split_and_combine(const fa::DecodeParams& p, int keys, int outer, voi
   // the bytes) or, for pages smaller than a stage, one page
   const uint32_t box = static_cast<uint32_t>(kPaged ? std::min(C::kT, keys) : C::kT);
   int rc;
-  if ((rc = encode_u8_4d(&tk, p.k, D, p.Hkv, keys, outer, box)) != FA_OK) return rc;
-  if ((rc = encode_u8_4d(&tv, p.v, D, p.Hkv, keys, outer, box)) != FA_OK) return rc;
-  auto kernel = fa::fa_decode_split_kernel<D, kPaged>;
-  if ((rc = ensure_smem_attr(kernel, C::kSmemBytes,
-                             g_attr_decode[(D == 128 ? 2 : 0) + (kPaged ? 1 : 0)])) != FA_OK)
-    return rc;
+  if ((rc = encode_u8_4d(&tk, p.k, C::kRow, p.Hkv, keys, outer, box)) != FA_OK) return rc;
+  if ((rc = encode_u8_4d(&tv, p.v, C::kRow, p.Hkv, keys, outer, box)) != FA_OK) return rc;
+  auto kernel = fa::fa_decode_split_kernel<D, kPaged, kBits>;
+  const int variant = (D == 128 ? 4 : 0) + (kPaged ? 2 : 0) + (kBits == 4 ? 1 : 0);
+  if ((rc = ensure_smem_attr(kernel, C::kSmemBytes, g_attr_decode[variant])) != FA_OK) return rc;
   dim3 grid(p.Hkv, p.splits, static_cast<unsigned>(gz));
   kernel<<<grid, 160, C::kSmemBytes, stream>>>(tk, tv, p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
@@ -224,28 +226,32 @@ int launch_split_and_combine(const fa::DecodeParams& p, int keys, int outer, voi
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-template <int D>
-int launch_decode(const void* q, const int8_t* k, const int8_t* v, const float* ks, const float* vs,
+template <int D, int kBits>
+int launch_decode(const void* q, const void* k, const void* v, const float* ks, const float* vs,
                   void* o, float* lse, int B, int Hq, int Hkv, int Skv, float scale, int splits,
                   void* ws, cudaStream_t stream) {
-  fa::DecodeParams p = decode_params(q, k, v, ks, vs, B, Hq, Hkv, D, scale, splits, ws);
+  fa::DecodeParams p = decode_params(q, static_cast<const int8_t*>(k),
+                                     static_cast<const int8_t*>(v), ks, vs, B, Hq, Hkv, D, scale,
+                                     splits, ws);
   p.Skv = Skv;
-  return launch_split_and_combine<D, false>(p, Skv, B, o, lse, stream);
+  return launch_split_and_combine<D, false, kBits>(p, Skv, B, o, lse, stream);
 }
 
-template <int D>
-int launch_decode_paged(const void* q, const int8_t* k, const int8_t* v, const float* ks,
+template <int D, int kBits>
+int launch_decode_paged(const void* q, const void* k, const void* v, const float* ks,
                         const float* vs, const int32_t* block_table, const int32_t* seqlens,
                         void* o, float* lse, int B, int Hq, int Hkv, int page_shift,
                         int max_pages, int num_pages, float scale, int splits, void* ws,
                         cudaStream_t stream) {
-  fa::DecodeParams p = decode_params(q, k, v, ks, vs, B, Hq, Hkv, D, scale, splits, ws);
+  fa::DecodeParams p = decode_params(q, static_cast<const int8_t*>(k),
+                                     static_cast<const int8_t*>(v), ks, vs, B, Hq, Hkv, D, scale,
+                                     splits, ws);
   p.block_table = block_table;
   p.seqlens = seqlens;
   p.max_pages = max_pages;
   p.num_pages = num_pages;
   p.page_shift = page_shift;
-  return launch_split_and_combine<D, true>(p, 1 << page_shift, num_pages, o, lse, stream);
+  return launch_split_and_combine<D, true, kBits>(p, 1 << page_shift, num_pages, o, lse, stream);
 }
 
 // Device address of g_noalloc_scratch on the current device.  In host code the symbol name is
@@ -280,6 +286,77 @@ __global__ void bounded_wait_selftest_kernel(uint64_t timeout_ns) {
   }
 }
 
+// Argument checks shared by the contiguous decode entry points.
+int check_decode(const void* q, const void* k, const void* v, const float* ks, const float* vs,
+                 const void* o, const float* lse, int B, int Hq, int Hkv, int Skv, int D,
+                 float scale, int num_splits) {
+  if (!q || !k || !v || !ks || !vs || !o) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Skv <= 0 || D <= 0 || num_splits <= 0)
+    return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(ks) ||
+      !aligned16(vs) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FA_ERR_ALIGNMENT;
+  return FA_OK;
+}
+
+int check_workspace(int B, int Hq, int D, int num_splits, const void* ws, size_t ws_bytes) {
+  if (!ws || ws_bytes < decode_ws_layout(B, Hq, D, num_splits, nullptr)) return FA_ERR_WORKSPACE;
+  return aligned16(ws) ? FA_OK : FA_ERR_ALIGNMENT;
+}
+
+int decode_contiguous(int bits, const void* q, const void* k, const void* v, const float* ks,
+                      const float* vs, void* o, float* lse, int B, int Hq, int Hkv, int Skv, int D,
+                      float scale, int splits, void* ws, cudaStream_t s) {
+  if (D == 128)
+    return bits == 8 ? launch_decode<128, 8>(q, k, v, ks, vs, o, lse, B, Hq, Hkv, Skv, scale,
+                                             splits, ws, s)
+                     : launch_decode<128, 4>(q, k, v, ks, vs, o, lse, B, Hq, Hkv, Skv, scale,
+                                             splits, ws, s);
+  return bits == 8
+             ? launch_decode<64, 8>(q, k, v, ks, vs, o, lse, B, Hq, Hkv, Skv, scale, splits, ws, s)
+             : launch_decode<64, 4>(q, k, v, ks, vs, o, lse, B, Hq, Hkv, Skv, scale, splits, ws, s);
+}
+
+int decode_paged(int bits, const void* q, const void* k, const void* v, const float* ks,
+                 const float* vs, const int32_t* block_table, const int32_t* seqlens, void* o,
+                 float* lse, int B, int Hq, int Hkv, int page_size, int max_pages, int num_pages,
+                 int D, float scale, int splits, void* ws, size_t ws_bytes, cudaStream_t st) {
+  if (!q || !k || !v || !ks || !vs || !block_table || !seqlens || !o) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || splits <= 0 || max_pages <= 0 || num_pages <= 0)
+    return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  int shift = -1;
+  for (int s = 4; s <= 16; ++s)
+    if (page_size == (1 << s)) shift = s;
+  if (shift < 0) return FA_ERR_INVALID_ARG;
+  if ((static_cast<long long>(max_pages) << shift) > (1ll << 30)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(ks) ||
+      !aligned16(vs) || (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
+      (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return FA_ERR_ALIGNMENT;
+  const int rc = check_workspace(B, Hq, D, splits, ws, ws_bytes);
+  if (rc != FA_OK) return rc;
+  if (D == 128)
+    return bits == 8 ? launch_decode_paged<128, 8>(q, k, v, ks, vs, block_table, seqlens, o, lse,
+                                                   B, Hq, Hkv, shift, max_pages, num_pages,
+                                                   scale, splits, ws, st)
+                     : launch_decode_paged<128, 4>(q, k, v, ks, vs, block_table, seqlens, o, lse,
+                                                   B, Hq, Hkv, shift, max_pages, num_pages,
+                                                   scale, splits, ws, st);
+  return bits == 8 ? launch_decode_paged<64, 8>(q, k, v, ks, vs, block_table, seqlens, o, lse, B,
+                                                Hq, Hkv, shift, max_pages, num_pages, scale,
+                                                splits, ws, st)
+                   : launch_decode_paged<64, 4>(q, k, v, ks, vs, block_table, seqlens, o, lse, B,
+                                                Hq, Hkv, shift, max_pages, num_pages, scale,
+                                                splits, ws, st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -304,29 +381,6 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
 size_t fa_decode_int8_workspace_bytes(int B, int Hq, int D, int num_splits) {
   if (B <= 0 || Hq <= 0 || D <= 0 || num_splits <= 0) return 0;
   return decode_ws_layout(B, Hq, D, num_splits, nullptr);
-}
-
-int fa_decode_int8(const void* q, const int8_t* k, const int8_t* v, const float* k_scale,
-                   const float* v_scale, void* o, float* lse, int B, int Hq, int Hkv, int Skv,
-                   int D, float scale, int num_splits, void* workspace, size_t workspace_bytes,
-                   void* stream) {
-  if (!q || !k || !v || !k_scale || !v_scale || !o) return FA_ERR_INVALID_ARG;
-  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Skv <= 0 || D <= 0 || num_splits <= 0)
-    return FA_ERR_INVALID_ARG;
-  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
-  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(k_scale) ||
-      !aligned16(v_scale) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
-    return FA_ERR_ALIGNMENT;
-  const size_t need = decode_ws_layout(B, Hq, D, num_splits, nullptr);
-  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return FA_ERR_ALIGNMENT;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return D == 128 ? launch_decode<128>(q, k, v, k_scale, v_scale, o, lse, B, Hq, Hkv, Skv, scale,
-                                       num_splits, workspace, s)
-                  : launch_decode<64>(q, k, v, k_scale, v_scale, o, lse, B, Hq, Hkv, Skv, scale,
-                                      num_splits, workspace, s);
 }
 
 const char* fa_status_string(int status) {
@@ -356,28 +410,39 @@ int fa_device_status(void* stream) {
   return (v & fa::kDevStatusBadIndex) ? FA_ERR_DEVICE_INDEX : FA_ERR_CUDA;
 }
 
+int fa_decode_int8(const void* q, const int8_t* k, const int8_t* v, const float* k_scale,
+                   const float* v_scale, void* o, float* lse, int B, int Hq, int Hkv, int Skv,
+                   int D, float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+  int rc = check_decode(q, k, v, k_scale, v_scale, o, lse, B, Hq, Hkv, Skv, D, scale, num_splits);
+  if (rc == FA_OK) rc = check_workspace(B, Hq, D, num_splits, workspace, workspace_bytes);
+  if (rc != FA_OK) return rc;
+  return decode_contiguous(8, q, k, v, k_scale, v_scale, o, lse, B, Hq, Hkv, Skv, D, scale,
+                           num_splits, workspace, static_cast<cudaStream_t>(stream));
+}
+
+int fa_decode_int4(const void* q, const uint8_t* k, const uint8_t* v, const float* k_scale,
+                   const float* v_scale, void* o, float* lse, int B, int Hq, int Hkv, int Skv,
+                   int D, float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+  int rc = check_decode(q, k, v, k_scale, v_scale, o, lse, B, Hq, Hkv, Skv, D, scale, num_splits);
+  if (rc == FA_OK) rc = check_workspace(B, Hq, D, num_splits, workspace, workspace_bytes);
+  if (rc != FA_OK) return rc;
+  return decode_contiguous(4, q, k, v, k_scale, v_scale, o, lse, B, Hq, Hkv, Skv, D, scale,
+                           num_splits, workspace, static_cast<cudaStream_t>(stream));
+}
+
 int fa_decode_int8_noalloc(const void* q, const int8_t* k, const int8_t* v, const float* k_scale,
                            const float* v_scale, void* o, float* lse, int B, int Hq, int Hkv,
                            int Skv, int D, float scale, int num_splits, void* stream) {
-  if (!q || !k || !v || !k_scale || !v_scale || !o) return FA_ERR_INVALID_ARG;
-  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Skv <= 0 || D <= 0 || num_splits <= 0)
-    return FA_ERR_INVALID_ARG;
-  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
-  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(k_scale) ||
-      !aligned16(v_scale) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
-    return FA_ERR_ALIGNMENT;
+  int rc = check_decode(q, k, v, k_scale, v_scale, o, lse, B, Hq, Hkv, Skv, D, scale, num_splits);
+  if (rc != FA_OK) return rc;
   if (decode_ws_layout(B, Hq, D, num_splits, nullptr) > FA_DECODE_INT8_NOALLOC_MAX_SCRATCH)
     return FA_ERR_WORKSPACE;
   void* ws = nullptr;
-  const int rc = noalloc_scratch_address(&ws);
-  if (rc != FA_OK) return rc;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return D == 128 ? launch_decode<128>(q, k, v, k_scale, v_scale, o, lse, B, Hq, Hkv, Skv, scale,
-                                       num_splits, ws, s)
-                  : launch_decode<64>(q, k, v, k_scale, v_scale, o, lse, B, Hq, Hkv, Skv, scale,
-                                      num_splits, ws, s);
+  if ((rc = noalloc_scratch_address(&ws)) != FA_OK) return rc;
+  return decode_contiguous(8, q, k, v, k_scale, v_scale, o, lse, B, Hq, Hkv, Skv, D, scale,
+                           num_splits, ws, static_cast<cudaStream_t>(stream));
 }
 
 int fa_decode_int8_paged(const void* q, const int8_t* k_pages, const int8_t* v_pages,
@@ -386,40 +451,20 @@ int fa_decode_int8_paged(const void* q, const int8_t* k_pages, const int8_t* v_p
                          int B, int Hq, int Hkv, int page_size, int max_pages_per_seq,
                          int num_pages, int D, float scale, int num_splits, void* workspace,
                          size_t workspace_bytes, void* stream) {
-  if (!q || !k_pages || !v_pages || !k_scale_pages || !v_scale_pages || !block_table ||
-      !seqlens || !o)
-    return FA_ERR_INVALID_ARG;
-  if (B <= 0 || Hq <= 0 || Hkv <= 0 || D <= 0 || num_splits <= 0 || max_pages_per_seq <= 0 ||
-      num_pages <= 0)
-    return FA_ERR_INVALID_ARG;
-  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
-  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
-  int page_shift = -1;
-  for (int s = 4; s <= 16; ++s)
-    if (page_size == (1 << s)) page_shift = s;
-  if (page_shift < 0) return FA_ERR_INVALID_ARG;
-  if ((static_cast<long long>(max_pages_per_seq) << page_shift) > (1ll << 30))
-    return FA_ERR_INVALID_ARG;
-  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
-  if (!aligned16(q) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(o) ||
-      !aligned16(k_scale_pages) || !aligned16(v_scale_pages) ||
-      (reinterpret_cast<uintptr_t>(block_table) & 3u) ||
-      (reinterpret_cast<uintptr_t>(seqlens) & 3u) ||
-      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
-    return FA_ERR_ALIGNMENT;
-  const size_t need = decode_ws_layout(B, Hq, D, num_splits, nullptr);
-  if (!workspace || workspace_bytes < need) return FA_ERR_WORKSPACE;
-  if (!aligned16(workspace)) return FA_ERR_ALIGNMENT;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return D == 128
-             ? launch_decode_paged<128>(q, k_pages, v_pages, k_scale_pages, v_scale_pages,
-                                        block_table, seqlens, o, lse, B, Hq, Hkv, page_shift,
-                                        max_pages_per_seq, num_pages, scale, num_splits,
-                                        workspace, st)
-             : launch_decode_paged<64>(q, k_pages, v_pages, k_scale_pages, v_scale_pages,
-                                       block_table, seqlens, o, lse, B, Hq, Hkv, page_shift,
-                                       max_pages_per_seq, num_pages, scale, num_splits,
-                                       workspace, st);
+  return decode_paged(8, q, k_pages, v_pages, k_scale_pages, v_scale_pages, block_table, seqlens,
+                      o, lse, B, Hq, Hkv, page_size, max_pages_per_seq, num_pages, D, scale,
+                      num_splits, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+int fa_decode_int4_paged(const void* q, const uint8_t* k_pages, const uint8_t* v_pages,
+                         const float* k_scale_pages, const float* v_scale_pages,
+                         const int32_t* block_table, const int32_t* seqlens, void* o, float* lse,
+                         int B, int Hq, int Hkv, int page_size, int max_pages_per_seq,
+                         int num_pages, int D, float scale, int num_splits, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  return decode_paged(4, q, k_pages, v_pages, k_scale_pages, v_scale_pages, block_table, seqlens,
+                      o, lse, B, Hq, Hkv, page_size, max_pages_per_seq, num_pages, D, scale,
+                      num_splits, workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 int fa_selftest_bounded_wait(int timeout_us, void* stream) {
