@@ -39,6 +39,9 @@ def lib():
         L.oracle_decode_int8_rows.argtypes = [_P] * 5 + [_I] * 5 + [_D, _I, _P, _L, _P, _P, _I]
         L.oracle_decode_int8_paged_rows.argtypes = [_P] * 7 + [_I] * 7 + [_D, _I, _P, _L, _P, _P, _I]
         L.oracle_decode_int8_paged_rows.restype = _I
+        L.oracle_attn_ext_rows.argtypes = ([_P, _P, _P] + [_I] * 6 + [_D, _I, _I, _I, _P, _L, _L]
+                                           + [_P, _L, _P, _P, _I])
+        L.oracle_attn_ext_rows.restype = _I
         L.oracle_unpack_int4.argtypes = [_P, _L, _P]
         L.oracle_unpack_int4.restype = _I
         for f in (L.oracle_attn_bf16_rows, L.oracle_attn_f64_rows, L.oracle_attn_brute,
@@ -215,3 +218,38 @@ def decode_int4_paged(q, kp4, vp4, ksp, vsp, block_table, seqlens, scale, num_sp
                       nthreads=0):
     return decode_int8_paged(q, unpack_int4(kp4), unpack_int4(vp4), ksp, vsp, block_table,
                              seqlens, scale, num_splits, nthreads)
+
+
+def attn_ext_rows(q, k, v, scale, causal, window, n_global, mask, rows, nthreads=0):
+    """Rows of the definition with an additive mask and global tokens.  q/k/v: bf16 bits;
+    mask: fp32 array broadcastable to [B, Hq, Sq, Skv] (leading dims of size 1 broadcast) or
+    None; rows: (n, 3) (b, h, i).  Returns (o [n, D], lse [n])."""
+    B, Hq, Hkv, Sq, Skv, D = _dims(q, k)
+    rows = np.ascontiguousarray(rows, dtype=np.int64).reshape(-1, 3)
+    n = rows.shape[0]
+    o = np.zeros((n, D))
+    lse = np.zeros(n)
+    q, k, v = (np.ascontiguousarray(t, dtype=np.uint16) for t in (q, k, v))
+    sb = sh = 0
+    mptr = None
+    if mask is not None:
+        mask = np.ascontiguousarray(mask, dtype=np.float32)
+        assert mask.ndim == 4 and mask.shape[2:] == (Sq, Skv)
+        assert mask.shape[0] in (1, B) and mask.shape[1] in (1, Hq)
+        sb = Sq * Skv * mask.shape[1] if mask.shape[0] == B else 0
+        sh = Sq * Skv if mask.shape[1] == Hq else 0
+        mptr = _ptr(mask)
+    rc = lib().oracle_attn_ext_rows(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Sq, Skv, D,
+                                    float(scale), int(causal), int(window), int(n_global), mptr,
+                                    sb, sh, _ptr(rows), n, _ptr(o), _ptr(lse), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_attn_ext_rows rejected its arguments")
+    return o, lse
+
+
+def attn_ext(q, k, v, scale, causal=0, window=0, n_global=0, mask=None, nthreads=0):
+    """Full output: (O [B,Sq,Hq,D], LSE [B,Hq,Sq])."""
+    B, Hq, Hkv, Sq, Skv, D = _dims(q, k)
+    o, lse = attn_ext_rows(q, k, v, scale, causal, window, n_global, mask, all_rows(B, Hq, Sq),
+                           nthreads)
+    return (o.reshape(B, Hq, Sq, D).transpose(0, 2, 1, 3).copy(), lse.reshape(B, Hq, Sq))

@@ -32,6 +32,15 @@
 //    dequantised values k_code * k_scale (exact in fp64), one query token per sequence.
 //    With num_splits > 1 it evaluates each key chunk separately and merges the partial
 //    results through their log-sum-exp, the same correction step the online softmax uses.
+//  * An additive mask tensor and global + local attention -- "FlashAttention variants: GQA,
+//    MQA, sparse attention", sliding-window section (the mask passed as atten_mask: -inf where a
+//    key is dropped, added to the scaled scores) and global+local section (a few global tokens
+//    attend to, and are attended by, every token; the others see their local window).  The
+//    printed global+local code concatenates two outputs along the sequence; the reading taken
+//    here is the union of the two key sets for each query, which is what merging the two
+//    partial results through their log-sum-exp gives.  `oracle_attn_ext_rows` adds
+//    M[b, h, i, j] (broadcast over b or h by a zero stride) to scale * q.k and, with G > 0
+//    global tokens, lets query i see key j when j < G or i < G besides the causal / window rule.
 //  * INT4 KV cache, the second format of the same KV-compression section ("INT8/INT4").  The
 //    pages give no packing; this project stores two 4-bit two's-complement codes per byte (dim
 //    2i in the low nibble, dim 2i+1 in the high nibble) with one fp32 scale per (token, KV head),
@@ -299,6 +308,66 @@ int oracle_attn_tiled(const double* q, const double* k, const double* v, int B, 
           *lrow = m[r] + std::log(l[r]);
         }
       }
+    }
+  }
+  return 0;
+}
+
+// The definition with an additive mask and global tokens, row by row, on bf16 inputs.
+// mask: fp32, element (b, h, i, j) at mask[b * mask_sb + h * mask_sh + i * Skv + j] (a zero
+// stride broadcasts), or null.  n_global = G >= 0.  Key j is visible to query i when the
+// causal / window rule admits it, or j < G, or i < G; its score is scale * q.k + mask, and a
+// score of -inf (from the mask) drops the key.
+int oracle_attn_ext_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
+                         int Hkv, int Sq, int Skv, int D, double scale, int causal, int window,
+                         int n_global, const float* mask, int64_t mask_sb, int64_t mask_sh,
+                         const int64_t* rows, int64_t nrows, double* o, double* lse,
+                         int nthreads) {
+  const Dims d{B, Hq, Hkv, Sq, Skv, D};
+  if (!dims_ok(d) || n_global < 0 || nrows < 0 || (nrows > 0 && (!rows || !o || !lse)))
+    return -1;
+  if (!q || !k || !v || mask_sb < 0 || mask_sh < 0) return -1;
+  for (int64_t r = 0; r < nrows; ++r) {
+    const int64_t b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+    if (b < 0 || b >= B || h < 0 || h >= Hq || i < 0 || i >= Sq) return -1;
+  }
+  if (nthreads <= 0) nthreads = omp_get_max_threads();
+#pragma omp parallel num_threads(nthreads)
+  {
+    std::vector<double> x(Skv);
+#pragma omp for schedule(dynamic, 4)
+    for (int64_t r = 0; r < nrows; ++r) {
+      const long b = rows[3 * r], h = rows[3 * r + 1], i = rows[3 * r + 2];
+      const long g = kv_head(d, h);
+      double* orow = o + r * D;
+      // scores of the visible keys, mask added
+      double m = kNegInf;
+      for (long j = 0; j < Skv; ++j) {
+        const bool vis = allowed(d, causal, window, i, j) ||
+                         (n_global > 0 && (j < n_global || i < n_global));
+        x[j] = kNegInf;
+        if (!vis) continue;
+        double dot = 0.0;
+        for (long t = 0; t < D; ++t)
+          dot += widen_bf16(q[q_index(d, b, i, h) + t]) * widen_bf16(k[kv_index(d, b, j, g) + t]);
+        x[j] = scale * dot;
+        if (mask) x[j] += static_cast<double>(mask[b * mask_sb + h * mask_sh + i * Skv + j]);
+        m = std::max(m, x[j]);
+      }
+      for (long t = 0; t < D; ++t) orow[t] = 0.0;
+      if (m == kNegInf) {
+        lse[r] = kNegInf;
+        continue;
+      }
+      double l = 0.0;
+      for (long j = 0; j < Skv; ++j) {
+        if (x[j] == kNegInf) continue;
+        const double pj = std::exp(x[j] - m);
+        l += pj;
+        for (long t = 0; t < D; ++t) orow[t] += pj * widen_bf16(v[kv_index(d, b, j, g) + t]);
+      }
+      for (long t = 0; t < D; ++t) orow[t] /= l;
+      lse[r] = m + std::log(l);
     }
   }
   return 0;
