@@ -97,6 +97,65 @@ def paged_decode_bytes(w, seqlens) -> int:
     return kv + 4 * pages + 4 * w.B + 2 * w.B * w.Hq * w.D * 2 + w.B * w.Hq * 4
 
 
+def time_calls(torch, stream, call, steps: int, warmup: int) -> float:
+    """Average ms per call of ``call`` over ``steps`` back-to-back launches (CUDA events)."""
+    for _ in range(warmup):
+        call()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        call()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / steps
+
+
+def global_local_flops(w, n_global: int) -> int:
+    """4*D flops per visible (query, key) pair under the causal window rule plus global tokens."""
+    import numpy as np
+    i = np.arange(w.Sq, dtype=np.int64)
+    ip = i + (w.Skv - w.Sq)
+    hi = np.minimum(ip, w.Skv - 1)
+    lo = np.maximum(0, ip - w.window + 1) if w.window > 0 else np.zeros_like(ip)
+    band = np.maximum(0, hi - lo + 1)
+    # keys below G outside the band, for rows that are not global themselves
+    extra = np.maximum(0, np.minimum(n_global, lo) - 0)
+    pairs = np.where(i < n_global, w.Skv, band + extra)
+    return int(pairs.sum()) * 4 * w.D * w.B * w.Hq
+
+
+def measure_mask_variants(fa, synthetic, torch, dev, stream, steps: int, warmup: int):
+    """The forward pass with a per-head additive bias mask on the MHA causal workload, and with
+    64 global tokens on the GQA sliding-window workload.  Returns {name: (ms, flops)}."""
+    import numpy as np
+    out = {}
+    w = synthetic.WORKLOADS["mha_causal"]
+    q, k, v = synthetic.make_qkv_torch(w, dev)
+    slopes = 2.0 ** (-8.0 * np.arange(1, w.Hq + 1) / w.Hq)
+    dist = (np.arange(w.Skv)[None, :] - np.arange(w.Sq)[:, None]).astype(np.float64)
+    mask = torch.from_numpy(
+        (slopes[:, None, None] * np.minimum(dist, 0.0)[None]).astype(np.float32)[None]).to(dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=dev)
+    ms = time_calls(torch, stream, lambda: fa.fa_fwd(q, k, v, causal=True, scale=w.scale, o=o,
+                                                      lse=lse, mask=mask, stream=stream),
+                    steps, warmup)
+    out["masked"] = (ms, prefill_flops(w))
+    del q, k, v, mask, o, lse
+    w = synthetic.WORKLOADS["gqa_sw512"]
+    q, k, v = synthetic.make_qkv_torch(w, dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=dev)
+    ms = time_calls(torch, stream, lambda: fa.fa_fwd(q, k, v, causal=True, window=w.window,
+                                                      scale=w.scale, o=o, lse=lse, n_global=64,
+                                                      stream=stream), steps, warmup)
+    out["global_local"] = (ms, global_local_flops(w, 64))
+    if fa.fa_device_status() != 0:
+        raise RuntimeError("a masked forward reported a device-side error")
+    return out
+
+
 def measure_paged_decode(fa, synthetic, torch, dev, stream, steps: int, warmup: int):
     """Time fa_decode_int8_paged on the paged workload (its own short loop after the step loop).
     Returns (ms per call averaged over ``steps`` launches, algorithmic bytes per call)."""
@@ -416,6 +475,9 @@ def main():
     i4_ms, i4_bytes = measure_int4_decode(fa, synthetic, torch, dev, stream,
                                           steps=min(K, 200), warmup=max(3, args.warmup // 4))
     i4_ms = max_over_ranks(i4_ms)
+    mv = measure_mask_variants(fa, synthetic, torch, dev, stream, steps=min(K, 100),
+                               warmup=max(3, args.warmup // 4))
+    mv = {kk: (max_over_ranks(ms), fl) for kk, (ms, fl) in mv.items()}
 
     # ---- end to end through the public API, host buffers, copies inside the timed region ----
     e2e = None
@@ -519,6 +581,21 @@ def main():
                 "unit": "GB/s", "peak": peaks["hbm_gbs"],
                 "frac": i4_bytes / (i4_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                 "launches": 2 * min(K, 200)},
+            "masked_prefill": {
+                "workload": "mha_causal (B=2, H=32, S=4096, D=128, causal) + per-head additive "
+                            "fp32 bias mask [1, 32, 4096, 4096]",
+                "kernel": "fa_prefill_kernel<128, mask>", "ms_per_call": mv["masked"][0],
+                "achieved": mv["masked"][1] / (mv["masked"][0] * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "frac": mv["masked"][1] / (mv["masked"][0] * 1e-3) / 1e12
+                        / peaks["bf16_tflops_sustained"]},
+            "global_local_prefill": {
+                "workload": "gqa_sw512 (B=3, Hq=32, Hkv=8, S=4096, D=128, causal window 512) + "
+                            "64 global tokens",
+                "kernel": "fa_prefill_kernel<128, global>", "ms_per_call": mv["global_local"][0],
+                "achieved": mv["global_local"][1] / (mv["global_local"][0] * 1e-3) / 1e12,
+                "unit": "TFLOP/s",
+                "frac": mv["global_local"][1] / (mv["global_local"][0] * 1e-3) / 1e12
+                        / peaks["bf16_tflops_sustained"]},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 3 * K,

@@ -85,6 +85,27 @@ FA_API int fa_fwd(const void* q, const void* k, const void* v, void* o, float* l
            int Hkv, int Sq, int Skv, int D, float scale, int causal, int window, void* stream);
 
 /*
+ * Forward pass with an additive mask tensor and / or global tokens, on top of fa_fwd's causal
+ * and window rule.  Sources: "FlashAttention variants: GQA, MQA, sparse attention",
+ * sliding-window section (the mask given as atten_mask, -inf where a key is dropped) and
+ * global+local section (a few global tokens attend to, and are attended by, every token).
+ *   n_global  >= 0.  Query i sees key j when the causal / window rule admits it, or j <
+ *             n_global, or i < n_global (global tokens are the first n_global positions of
+ *             both the query and the key sequence).  Key tiles no query of a block needs are
+ *             never loaded.
+ *   mask      fp32 or NULL: element (b, h, i, j) at mask[b * mask_batch_stride + h *
+ *             mask_head_stride + i * Skv + j], added to scale * q.k; -inf drops the key.  A zero
+ *             stride broadcasts over batch or heads.  16-byte aligned; rows are read with vector
+ *             loads when Skv and both strides are multiples of 4.
+ * Every other argument is that of fa_fwd; fa_fwd(...) is fa_fwd_ext(..., 0, NULL, 0, 0, ...).
+ * A row whose every key is dropped gets O = 0 and LSE = -inf.
+ */
+FA_API int fa_fwd_ext(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                      int Hq, int Hkv, int Sq, int Skv, int D, float scale, int causal,
+                      int window, int n_global, const float* mask, int64_t mask_batch_stride,
+                      int64_t mask_head_stride, void* stream);
+
+/*
  * Bytes of device workspace fa_decode_int8 needs: fp32 partial outputs [num_splits, B, Hq, D]
  * followed by fp32 partial log-sum-exps [num_splits, B, Hq], padded to 256 bytes.
  * Returns 0 for invalid sizes.

@@ -32,7 +32,7 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("fa_fwd", "fa_decode_int8", "fa_decode_int8_workspace_bytes", "fa_status_string",
               "fa_device_status", "fa_selftest_bounded_wait", "fa_decode_int8_noalloc",
-              "fa_decode_int8_paged", "fa_decode_int4", "fa_decode_int4_paged"):
+              "fa_decode_int8_paged", "fa_decode_int4", "fa_decode_int4_paged", "fa_fwd_ext"):
         assert n in names
 
 
@@ -78,6 +78,22 @@ def fwd(L, q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, Hq=2, Hkv=2, Sq=128, S
 ])
 def test_fwd_rejects(L, kw, code):
     assert fwd(L, **kw) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_global=-1), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(sb=-4), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(mask=FAKE + 4), fa.STATUS["FA_ERR_ALIGNMENT"]),
+    (dict(window=8), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(D=32), fa.STATUS["FA_ERR_UNSUPPORTED"]),
+])
+def test_fwd_ext_rejects(L, kw, code):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=None, B=1, Hq=2, Hkv=2, Sq=128, Skv=128, D=64,
+             scale=0.125, causal=0, window=0, n_global=0, mask=FAKE, sb=0, sh=0)
+    a.update(kw)
+    assert L.fa_fwd_ext(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"],
+                        a["Sq"], a["Skv"], a["D"], a["scale"], a["causal"], a["window"],
+                        a["n_global"], a["mask"], a["sb"], a["sh"], None) == code
 
 
 def dec(L, q=FAKE, k=FAKE, v=FAKE, ks=FAKE, vs=FAKE, o=FAKE, lse=None, B=2, Hq=8, Hkv=2, Skv=100,

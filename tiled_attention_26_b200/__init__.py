@@ -54,6 +54,9 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         L.fa_fwd.argtypes = [_P, _P, _P, _P, _P] + [_I] * 6 + [_F, _I, _I, _P]
         L.fa_fwd.restype = _I
+        L.fa_fwd_ext.argtypes = ([_P, _P, _P, _P, _P] + [_I] * 6 + [_F, _I, _I, _I, _P,
+                                 ctypes.c_int64, ctypes.c_int64, _P])
+        L.fa_fwd_ext.restype = _I
         L.fa_decode_int8_workspace_bytes.argtypes = [_I, _I, _I, _I]
         L.fa_decode_int8_workspace_bytes.restype = _Z
         L.fa_decode_int8.argtypes = [_P] * 7 + [_I] * 5 + [_F, _I, _P, _Z, _P]
@@ -100,8 +103,12 @@ def _check(t, name, dtype, shape, device):
 
 
 def fa_fwd(q, k, v, causal: bool = False, window: int = 0, scale: float | None = None,
-           o=None, lse=None, return_lse: bool = True, stream=None):
+           o=None, lse=None, return_lse: bool = True, stream=None, n_global: int = 0,
+           mask=None):
     """Attention forward.  q: bf16 [B, Sq, Hq, D] on CUDA; k, v: bf16 [B, Skv, Hkv, D].
+    ``n_global``: the first n_global positions attend to, and are attended by, every position.
+    ``mask``: optional fp32 additive mask [Bm, Hm, Sq, Skv] with Bm in {1, B}, Hm in {1, Hq}
+    (size-1 dims broadcast), added to scale * q.k; -inf drops a key.
 
     Returns ``(o, lse)``: o bf16 [B, Sq, Hq, D], lse fp32 [B, Hq, Sq] (natural log; None when
     ``return_lse`` is false and no ``lse`` buffer is given)."""
@@ -123,9 +130,18 @@ def fa_fwd(q, k, v, causal: bool = False, window: int = 0, scale: float | None =
         _check(lse, "lse", torch.float32, (B, Hq, Sq), dev)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                      lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Sq, Skv, D,
-                      float(scale), int(bool(causal)), int(window), _stream_ptr(stream))
+    sb = sh = 0
+    if mask is not None:
+        if mask.dim() != 4 or mask.shape[0] not in (1, B) or mask.shape[1] not in (1, Hq):
+            raise ValueError("mask must be [1 or B, 1 or Hq, Sq, Skv]")
+        _check(mask, "mask", torch.float32, (mask.shape[0], mask.shape[1], Sq, Skv), dev)
+        sh = Sq * Skv if mask.shape[1] == Hq else 0
+        sb = Sq * Skv * mask.shape[1] if mask.shape[0] == B else 0
+    rc = lib().fa_fwd_ext(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                          lse.data_ptr() if lse is not None else None, B, Hq, Hkv, Sq, Skv, D,
+                          float(scale), int(bool(causal)), int(window), int(n_global),
+                          mask.data_ptr() if mask is not None else None, sb, sh,
+                          _stream_ptr(stream))
     if rc != 0:
         raise FaError(rc, "fa_fwd")
     return o, lse

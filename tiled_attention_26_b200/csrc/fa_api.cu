@@ -92,12 +92,20 @@ int ensure_smem_attr(Kernel kernel, int bytes, std::atomic<uint64_t>& done_mask)
   return FA_OK;
 }
 
-std::atomic<uint64_t> g_attr_prefill64{0}, g_attr_prefill128{0};
+std::atomic<uint64_t> g_attr_prefill[8];
+std::atomic<int> g_prefill_regs[8] = {};  // registers per thread of each variant, 0 = not read
 
-template <int D>
+// The optional parts of a forward call: an additive mask and global tokens.
+struct PrefillExtra {
+  const float* mask = nullptr;
+  long long mask_sb = 0, mask_sh = 0;
+  int n_global = 0;
+};
+
+template <int D, int kMode>
 int launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                    int Hkv, int Sq, int Skv, float scale, int causal, int window,
-                   cudaStream_t stream) {
+                   const PrefillExtra& ex, cudaStream_t stream) {
   using C = fa::PrefillCfg<D>;
   fa::PrefillParams p{};
   p.B = B;
@@ -116,6 +124,12 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
   p.window = window;
   p.lse = lse;
   p.timeout_ns = kKernelTimeoutNs;
+  p.mask = ex.mask;
+  p.mask_sb = ex.mask_sb;
+  p.mask_sh = ex.mask_sh;
+  p.inv_scale = 1.0f / scale;
+  p.mask_vec = (Skv % 4 == 0 && ex.mask_sb % 4 == 0 && ex.mask_sh % 4 == 0) ? 1 : 0;
+  p.n_global = ex.n_global;
 
   const long long grid = static_cast<long long>(p.n_qblocks) * B * Hkv * p.NP;
   if (grid <= 0 || grid > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
@@ -128,18 +142,17 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
   if ((rc = encode_bf16_4d(&tv, v, D, Hkv, Skv, B, 1, 128)) != FA_OK) return rc;
   if ((rc = encode_bf16_4d(&to, o, D, Hq, Sq, B, p.Gp, tpt)) != FA_OK) return rc;
 
-  auto kernel = fa::fa_prefill_kernel<D>;
-  if ((rc = ensure_smem_attr(kernel, C::kSmemBytes,
-                             D == 128 ? g_attr_prefill128 : g_attr_prefill64)) != FA_OK)
-    return rc;
+  auto kernel = fa::fa_prefill_kernel<D, kMode>;
+  const int variant = (D == 128 ? 4 : 0) + kMode;
+  if ((rc = ensure_smem_attr(kernel, C::kSmemBytes, g_attr_prefill[variant])) != FA_OK) return rc;
   // The kernel redistributes its launch registers between warpgroups (setmaxnreg); that only
   // completes if the launch gave every thread at least kMinLaunchRegs.
-  static int launch_regs[2] = {-1, -1};
-  int& regs = launch_regs[D == 128 ? 1 : 0];
-  if (regs < 0) {
+  int regs = g_prefill_regs[variant].load(std::memory_order_acquire);
+  if (regs == 0) {
     cudaFuncAttributes attr;
     if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return FA_ERR_CUDA;
     regs = attr.numRegs;
+    g_prefill_regs[variant].store(regs, std::memory_order_release);
   }
   if (regs < C::kMinLaunchRegs) return FA_ERR_UNSUPPORTED;
   kernel<<<static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, to, p);
@@ -361,21 +374,49 @@ int decode_paged(int bits, const void* q, const void* k, const void* v, const fl
 
 extern "C" {
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
-           int Sq, int Skv, int D, float scale, int causal, int window, void* stream) {
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+           int Hkv, int Sq, int Skv, int D, float scale, int causal, int window, void* stream) {
+  return fa_fwd_ext(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, D, scale, causal, window, 0, nullptr, 0,
+                    0, stream);
+}
+
+int fa_fwd_ext(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+               int Hkv, int Sq, int Skv, int D, float scale, int causal, int window,
+               int n_global, const float* mask, int64_t mask_batch_stride,
+               int64_t mask_head_stride, void* stream) {
   if (!q || !k || !v || !o) return FA_ERR_INVALID_ARG;
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq <= 0 || Skv <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
   if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
   if (window < 0 || (window > 0 && !causal)) return FA_ERR_INVALID_ARG;
+  if (n_global < 0 || mask_batch_stride < 0 || mask_head_stride < 0) return FA_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) ||
-      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) ||
+      (mask && (reinterpret_cast<uintptr_t>(mask) & 15u)))
     return FA_ERR_ALIGNMENT;
+  PrefillExtra ex;
+  ex.mask = mask;
+  ex.mask_sb = mask_batch_stride;
+  ex.mask_sh = mask_head_stride;
+  ex.n_global = n_global;
+  const int mode = (mask ? fa::kModeMask : 0) | (n_global > 0 ? fa::kModeGlobal : 0);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return D == 128 ? launch_prefill<128>(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, window, s)
-                  : launch_prefill<64>(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, window, s);
+#define FA_PREFILL_CASE(DD, MM)                                                                 \
+  if (D == DD && mode == MM)                                                                   \
+    return launch_prefill<DD, MM>(q, k, v, o, lse, B, Hq, Hkv, Sq, Skv, scale, causal, window, \
+                                  ex, s);
+  FA_PREFILL_CASE(128, 0)
+  FA_PREFILL_CASE(128, 1)
+  FA_PREFILL_CASE(128, 2)
+  FA_PREFILL_CASE(128, 3)
+  FA_PREFILL_CASE(64, 0)
+  FA_PREFILL_CASE(64, 1)
+  FA_PREFILL_CASE(64, 2)
+  FA_PREFILL_CASE(64, 3)
+#undef FA_PREFILL_CASE
+  return FA_ERR_UNSUPPORTED;
 }
 
 size_t fa_decode_int8_workspace_bytes(int B, int Hq, int D, int num_splits) {

@@ -46,7 +46,33 @@ struct PrefillParams {
   int window;  // <= 0: none
   float* lse;  // [B, Hq, Sq] natural log, may be null
   uint64_t timeout_ns;
+  // additive mask (kModeMask): fp32, element (b, h, i, j) at mask[b*mask_sb + h*mask_sh +
+  // i*Skv + j]; a zero stride broadcasts
+  const float* mask;
+  long long mask_sb, mask_sh;
+  float inv_scale;  // 1 / scale: the mask joins the raw scores as mask / scale
+  int mask_vec;     // every mask row starts 16-byte aligned (Skv and both strides % 4 == 0)
+  int n_global;     // kModeGlobal: tokens [0, n_global) attend to and are attended by all
 };
+
+// The key tiles one Q tile needs: [first, last], restricted (with global tokens and no global
+// query in the tile) to the global tiles [0, gT) and the band [jlo, jhi).
+struct TileSet {
+  int first, last, jlo, jhi;
+  bool allq;  // the tile holds a global query: every key tile
+  template <bool kGlobal>
+  __device__ __forceinline__ bool has(int j, int gT) const {
+    if (j < first || j > last) return false;
+    if (!kGlobal || allq) return true;
+    return j < gT || (j >= jlo && j < jhi);
+  }
+};
+
+// Kernel variants: an additive mask tensor, and global tokens on top of the causal / window
+// rule ("FlashAttention variants: GQA, MQA, sparse attention", sliding-window section: the
+// mask passed as atten_mask; global+local section).
+constexpr int kModeMask = 1;
+constexpr int kModeGlobal = 2;
 
 template <int D>
 struct PrefillCfg {
@@ -156,7 +182,7 @@ __device__ __forceinline__ void exp_half(const uint32_t (&sv)[4][32], int half, 
   tmem_st32(taddr + 32 * half, pk);
 }
 
-template <int D>
+template <int D, int kMode>
 __global__ void __launch_bounds__(384, 1)
     fa_prefill_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_k,
@@ -176,9 +202,15 @@ __global__ void __launch_bounds__(384, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- work item: heaviest (last) query blocks first ----
+  // ---- work item: heaviest query blocks first: the blocks holding global queries (they see
+  // every key), then the rest from the last block (the longest causal rows) down ----
   const int per_qb = p.B * p.Hkv * p.NP;
-  const int qb = p.n_qblocks - 1 - static_cast<int>(blockIdx.x) / per_qb;
+  const int order = static_cast<int>(blockIdx.x) / per_qb;
+  int qb = p.n_qblocks - 1 - order;
+  if constexpr ((kMode & kModeGlobal) != 0) {
+    const int n_gqb = min(p.n_qblocks, (p.n_global + 256 / p.Gp - 1) / (256 / p.Gp));
+    qb = order < n_gqb ? order : p.n_qblocks - 1 - (order - n_gqb);
+  }
   int rem = static_cast<int>(blockIdx.x) % per_qb;
   const int b = rem / (p.Hkv * p.NP);
   rem %= p.Hkv * p.NP;
@@ -206,9 +238,42 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
   }
-  const bool act0 = jhi[0] > jlo[0], act1 = jhi[1] > jlo[1];
-  const int J0 = act0 ? (act1 ? min(jlo[0], jlo[1]) : jlo[0]) : (act1 ? jlo[1] : 0);
-  const int J1 = act0 ? (act1 ? max(jhi[0], jhi[1]) : jhi[0]) : (act1 ? jhi[1] : 0);
+  // Key tiles each Q tile needs.  Without global tokens: the contiguous band [jlo, jhi).  With
+  // G global tokens: the tiles holding keys [0, G) plus the band, or every tile when the Q
+  // tile holds a global query; the tiles in between are never loaded.
+  constexpr bool kGlobal = (kMode & kModeGlobal) != 0;
+  constexpr bool kMask = (kMode & kModeMask) != 0;
+  const int nK = (p.Skv + 127) / 128;
+  const int gT = kGlobal ? min(nK, (p.n_global + 127) / 128) : 0;
+  TileSet ts[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int first = tok0 + t * tpt;
+    ts[t] = TileSet{jlo[t], jhi[t] - 1, jlo[t], jhi[t], false};
+    if (kGlobal && first < p.Sq) {
+      ts[t].allq = first < p.n_global;
+      if (ts[t].allq) {
+        ts[t].first = 0;
+        ts[t].last = nK - 1;
+      } else if (gT > 0) {
+        ts[t].first = 0;
+        ts[t].last = max(gT - 1, jhi[t] - 1);
+      }
+    }
+  }
+  const TileSet ts0 = ts[0], ts1 = ts[1];
+  auto part = [&](int t, int j) -> bool { return (t ? ts1 : ts0).has<kGlobal>(j, gT); };
+  const bool act0 = ts0.last >= ts0.first, act1 = ts1.last >= ts1.first;
+  const int J0 = act0 ? (act1 ? min(ts0.first, ts1.first) : ts0.first) : (act1 ? ts1.first : 0);
+  const int J1 = act0 ? (act1 ? max(ts0.last, ts1.last) : ts0.last) + 1 : (act1 ? ts1.last + 1 : 0);
+  auto need = [&](int j) { return part(0, j) || part(1, j); };
+  // next tile after j that some Q tile needs (J1 if none)
+  auto next_need = [&](int j) {
+    int x = j + 1;
+    if constexpr (kGlobal)
+      while (x < J1 && !need(x)) ++x;
+    return x;
+  };
 
   // ---- setup ----
   if (threadIdx.x == 0) {
@@ -252,10 +317,11 @@ __global__ void __launch_bounds__(384, 1)
           tma_load_4d(sQ + t * C::kTileBytes + hf * C::kAtomBytes, &tm_q, bar(C::kBarQ), 64 * hf,
                       h0, tok0 + t * tpt, b);
       bool ok = true;
-      for (int j = J0; j < J1 && ok; ++j) {
+      int kt = 0;  // index of tile j among the needed tiles
+      for (int j = J0; j < J1 && ok; j = next_need(j), ++kt) {
 #pragma unroll
         for (int kind = 0; kind < 2; ++kind) {
-          const int pos = 2 * (j - J0) + kind;
+          const int pos = 2 * kt + kind;
           const int s = pos % C::kStages;
           if (!mbar_wait(bar(C::kBarKVEmpty + s), ((pos / C::kStages) & 1) ^ 1, ctl)) {
             ok = false;
@@ -322,7 +388,6 @@ __global__ void __launch_bounds__(384, 1)
         tc_fence_after();
         return ok;
       };
-      auto part = [&](int t, int j) { return j >= jlo[t] && j < jhi[t]; };
       int n[2] = {0, 0};
       bool ok = mbar_wait(bar(C::kBarQ), 0, ctl);
       if (ok && J1 > J0) {
@@ -336,31 +401,33 @@ __global__ void __launch_bounds__(384, 1)
             }
           tc_commit(bar(C::kBarKVEmpty + 0));
         }
-        for (int j = J0; j < J1 && ok; ++j) {
-          const int vpos = 2 * (j - J0) + 1, kpos = vpos + 1;
+        int kt = 0;
+        for (int j = J0, jn; j < J1 && ok; j = jn, ++kt) {
+          jn = next_need(j);
+          const int vpos = 2 * kt + 1, kpos = vpos + 1;
           const int vslot = vpos % C::kStages, kslot = kpos % C::kStages;
-          const bool nxt = j + 1 < J1;
+          const bool nxt = jn < J1;
           if (!(ok = kv_wait(vpos))) break;
           if (part(0, j)) {
-            if (!(ok = issue_pv(0, vslot, j == jlo[0], n[0] & 1))) break;
+            if (!(ok = issue_pv(0, vslot, j == ts0.first, n[0] & 1))) break;
             ++n[0];
-            if (j == jhi[0] - 1) tc_commit(bar(C::kBarOFinal + 0));
+            if (j == ts0.last) tc_commit(bar(C::kBarOFinal + 0));
           }
           if (nxt) {
             if (!(ok = kv_wait(kpos))) break;
-            if (part(0, j + 1)) {
+            if (part(0, jn)) {
               issue_qk(0, kslot);
               tc_commit(bar(C::kBarSFull + 0));
             }
           }
           if (part(1, j)) {
-            if (!(ok = issue_pv(1, vslot, j == jlo[1], n[1] & 1))) break;
+            if (!(ok = issue_pv(1, vslot, j == ts1.first, n[1] & 1))) break;
             ++n[1];
-            if (j == jhi[1] - 1) tc_commit(bar(C::kBarOFinal + 1));
+            if (j == ts1.last) tc_commit(bar(C::kBarOFinal + 1));
           }
           tc_commit(bar(C::kBarKVEmpty + vslot));
           if (nxt) {
-            if (part(1, j + 1)) {
+            if (part(1, jn)) {
               issue_qk(1, kslot);
               tc_commit(bar(C::kBarSFull + 1));
             }
@@ -380,7 +447,7 @@ __global__ void __launch_bounds__(384, 1)
     // ================= softmax + correction + epilogue =================
     const int t = warp >> 2;
     const int r = threadIdx.x & 127;
-    const int t_jlo = t ? jlo[1] : jlo[0], t_jhi = t ? jhi[1] : jhi[0];
+    const TileSet my_ts = t ? ts1 : ts0;
     const int t_lo_last = t ? lo_last[1] : lo_last[0];
     const int t_hi_first = t ? hi_first[1] : hi_first[0];
     const uint32_t colS = t ? C::colS(1) : C::colS(0);
@@ -390,10 +457,19 @@ __global__ void __launch_bounds__(384, 1)
     const int i = tok0 + R / p.Gp;
     const int hh = h0 + R % p.Gp;
     const int my_lo = vis_lo(p, i), my_hi = vis_hi(p, i);
+    const int t_last_tok = min(tok0 + t * tpt + tpt, p.Sq) - 1;
     const float sl2 = p.scale_log2;
+    // this row's mask, or null (no mask, or a padding row past Sq)
+    const float* mrow = nullptr;
+    if constexpr (kMask)
+      if (i < p.Sq)
+        mrow = p.mask + b * p.mask_sb + hh * p.mask_sh + static_cast<long long>(i) * p.Skv;
+    const bool mvec = p.mask_vec != 0;  // rows start 16-byte aligned: vector loads
     float m = -INFINITY, l = 0.f;
     int n = 0;
-    for (int j = t_jlo; j < t_jhi; ++j) {
+    for (int j = my_ts.first; j <= my_ts.last; ++j) {
+      if constexpr (kGlobal)
+        if (!my_ts.has<kGlobal>(j, gT)) continue;
       bool ok = mbar_wait(bar(C::kBarSFull + t), n & 1, ctl);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
@@ -401,14 +477,48 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(trow + colS + 32 * c, sv[c]);
       tmem_wait_ld();
-      const bool need_mask = (128 * j < t_lo_last) || (128 * j + 127 > t_hi_first);
+      if constexpr (kMask) {
+        // scores += mask / scale (the exponent then carries scale * s + mask, in log2 units)
+        if (mrow != nullptr) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int q4 = 0; q4 < 8; ++q4) {
+              const int key = 128 * j + 32 * c + 4 * q4;
+              float mv[4] = {0.f, 0.f, 0.f, 0.f};
+              if (mvec) {
+                if (key < p.Skv) {
+                  const float4 x = __ldg(reinterpret_cast<const float4*>(mrow + key));
+                  mv[0] = x.x; mv[1] = x.y; mv[2] = x.z; mv[3] = x.w;
+                }
+              } else {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  if (key + e < p.Skv) mv[e] = __ldg(mrow + key + e);
+              }
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                sv[c][4 * q4 + e] = __float_as_uint(
+                    fmaf(mv[e], p.inv_scale, __uint_as_float(sv[c][4 * q4 + e])));
+            }
+        }
+      }
+      bool need_mask = (128 * j < t_lo_last) || (128 * j + 127 > t_hi_first);
+      if constexpr (kGlobal) {
+        const bool full = (128 * j + 127 < p.Skv) &&
+                          (t_last_tok < p.n_global || 128 * j + 127 < p.n_global || !need_mask);
+        need_mask = !full;
+      }
       if (need_mask) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int k = 0; k < 32; ++k) {
             const int key = 128 * j + 32 * c + k;
-            if (key < my_lo || key > my_hi) sv[c][k] = __float_as_uint(-INFINITY);
+            bool vis = key >= my_lo && key <= my_hi;
+            if constexpr (kGlobal)
+              vis = vis || (key < p.Skv && (key < p.n_global || i < p.n_global));
+            if (!vis) sv[c][k] = __float_as_uint(-INFINITY);
           }
       }
       const float m_tile = row_max128(sv) * sl2;
@@ -444,7 +554,7 @@ __global__ void __launch_bounds__(384, 1)
       uint64_t acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        if (need_mask) {
+        if (need_mask || kMask) {
           exp_half<false>(sv, half, sl2, m_use, trow + colS, acc0, acc1);
         } else {
           exp_half<true>(sv, half, sl2, m_use, trow + colS, acc0, acc1);
