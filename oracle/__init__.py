@@ -42,6 +42,8 @@ def lib():
         L.oracle_attn_ext_rows.argtypes = ([_P, _P, _P] + [_I] * 6 + [_D, _I, _I, _I, _P, _L, _L]
                                            + [_P, _L, _P, _P, _I])
         L.oracle_attn_ext_rows.restype = _I
+        L.oracle_attn_bwd.argtypes = [_P] * 4 + [_I] * 6 + [_D, _I, _I, _P, _P, _P, _I]
+        L.oracle_attn_bwd.restype = _I
         L.oracle_unpack_int4.argtypes = [_P, _L, _P]
         L.oracle_unpack_int4.restype = _I
         for f in (L.oracle_attn_bf16_rows, L.oracle_attn_f64_rows, L.oracle_attn_brute,
@@ -253,3 +255,19 @@ def attn_ext(q, k, v, scale, causal=0, window=0, n_global=0, mask=None, nthreads
     o, lse = attn_ext_rows(q, k, v, scale, causal, window, n_global, mask, all_rows(B, Hq, Sq),
                            nthreads)
     return (o.reshape(B, Hq, Sq, D).transpose(0, 2, 1, 3).copy(), lse.reshape(B, Hq, Sq))
+
+
+def attn_bwd(q, k, v, dout, scale, causal=0, window=0, nthreads=0):
+    """Gradients (dQ [B,Sq,Hq,D], dK, dV [B,Skv,Hkv,D]) of sum(dout * O) for the definition, in
+    fp64, from bf16 bit patterns."""
+    B, Hq, Hkv, Sq, Skv, D = _dims(q, k)
+    q, k, v, dout = (np.ascontiguousarray(t, dtype=np.uint16) for t in (q, k, v, dout))
+    dq = np.zeros((B, Sq, Hq, D))
+    dk = np.zeros((B, Skv, Hkv, D))
+    dv = np.zeros((B, Skv, Hkv, D))
+    rc = lib().oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), B, Hq, Hkv, Sq, Skv, D,
+                               float(scale), int(causal), int(window), _ptr(dq), _ptr(dk),
+                               _ptr(dv), int(nthreads))
+    if rc != 0:
+        raise ValueError("oracle_attn_bwd rejected its arguments")
+    return dq, dk, dv

@@ -32,6 +32,12 @@
 //    dequantised values k_code * k_scale (exact in fp64), one query token per sequence.
 //    With num_splits > 1 it evaluates each key chunk separately and merges the partial
 //    results through their log-sum-exp, the same correction step the online softmax uses.
+//  * The backward pass -- "FlashAttention on Ascend NPUs", recomputation section: the attention
+//    matrix is not stored; the backward pass recomputes it.  `oracle_attn_bwd` differentiates
+//    L = sum(dO * O) through the definition for one (b, h) at a time with the probabilities of
+//    the visible keys written out: D_i = sum_t dO_it O_it, dV_j = sum_i P_ij dO_i,
+//    dP_ij = dO_i . v_j, dS_ij = P_ij (dP_ij - D_i), dQ_i = scale sum_j dS_ij k_j,
+//    dK_j = scale sum_i dS_ij q_i; GQA sums dK, dV over the query heads of a KV head.
 //  * An additive mask tensor and global + local attention -- "FlashAttention variants: GQA,
 //    MQA, sparse attention", sliding-window section (the mask passed as atten_mask: -inf where a
 //    key is dropped, added to the scaled scores) and global+local section (a few global tokens
@@ -368,6 +374,83 @@ int oracle_attn_ext_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v
       }
       for (long t = 0; t < D; ++t) orow[t] /= l;
       lse[r] = m + std::log(l);
+    }
+  }
+  return 0;
+}
+
+// Gradients of the definition (causal / window rule) on bf16 inputs: q, do [B,Sq,Hq,D];
+// k, v [B,Skv,Hkv,D].  Outputs fp64: dq [B,Sq,Hq,D], dk, dv [B,Skv,Hkv,D] (overwritten).
+// P is recomputed exactly from the scores; O and D come from the same exact P.
+int oracle_attn_bwd(const uint16_t* q, const uint16_t* k, const uint16_t* v, const uint16_t* dout,
+                    int B, int Hq, int Hkv, int Sq, int Skv, int D, double scale, int causal,
+                    int window, double* dq, double* dk, double* dv, int nthreads) {
+  const Dims d{B, Hq, Hkv, Sq, Skv, D};
+  if (!dims_ok(d) || !q || !k || !v || !dout || !dq || !dk || !dv) return -1;
+  const size_t nq = static_cast<size_t>(B) * Sq * Hq * D, nk = static_cast<size_t>(B) * Skv * Hkv * D;
+  for (size_t t = 0; t < nq; ++t) dq[t] = 0.0;
+  for (size_t t = 0; t < nk; ++t) dk[t] = dv[t] = 0.0;
+  if (nthreads <= 0) nthreads = omp_get_max_threads();
+  const long G = Hq / Hkv;
+  // one task per (b, KV head): its query heads write disjoint dq rows and share dk, dv rows
+#pragma omp parallel for num_threads(nthreads) schedule(dynamic, 1)
+  for (long task = 0; task < static_cast<long>(B) * Hkv; ++task) {
+    const long b = task / Hkv, g = task % Hkv;
+    std::vector<double> P(static_cast<size_t>(Sq) * Skv), dS(static_cast<size_t>(Sq) * Skv);
+    std::vector<double> Orow(D);
+    for (long h = g * G; h < (g + 1) * G; ++h) {
+      for (long i = 0; i < Sq; ++i) {
+        // probabilities of row i (0 where a key is not visible)
+        double* prow = P.data() + i * Skv;
+        double m = kNegInf;
+        for (long j = 0; j < Skv; ++j) {
+          prow[j] = kNegInf;
+          if (!allowed(d, causal, window, i, j)) continue;
+          double dot = 0.0;
+          for (long t = 0; t < D; ++t)
+            dot += widen_bf16(q[q_index(d, b, i, h) + t]) * widen_bf16(k[kv_index(d, b, j, g) + t]);
+          prow[j] = scale * dot;
+          m = std::max(m, prow[j]);
+        }
+        double l = 0.0;
+        for (long j = 0; j < Skv; ++j) {
+          prow[j] = (prow[j] == kNegInf) ? 0.0 : std::exp(prow[j] - m);
+          l += prow[j];
+        }
+        for (long j = 0; j < Skv; ++j) prow[j] = (l > 0.0) ? prow[j] / l : 0.0;
+        // O_i and D_i = dO_i . O_i
+        for (long t = 0; t < D; ++t) Orow[t] = 0.0;
+        for (long j = 0; j < Skv; ++j)
+          if (prow[j] != 0.0)
+            for (long t = 0; t < D; ++t) Orow[t] += prow[j] * widen_bf16(v[kv_index(d, b, j, g) + t]);
+        double Di = 0.0;
+        for (long t = 0; t < D; ++t) Di += widen_bf16(dout[q_index(d, b, i, h) + t]) * Orow[t];
+        // dS_ij = P_ij (dO_i . v_j - D_i)
+        for (long j = 0; j < Skv; ++j) {
+          double dp = 0.0;
+          if (prow[j] != 0.0)
+            for (long t = 0; t < D; ++t)
+              dp += widen_bf16(dout[q_index(d, b, i, h) + t]) * widen_bf16(v[kv_index(d, b, j, g) + t]);
+          dS[i * Skv + j] = prow[j] * (dp - Di);
+        }
+      }
+      // dV_j += sum_i P_ij dO_i ; dK_j += scale sum_i dS_ij q_i ; dQ_i = scale sum_j dS_ij k_j
+      for (long j = 0; j < Skv; ++j)
+        for (long i = 0; i < Sq; ++i) {
+          const double pij = P[i * Skv + j], sij = dS[i * Skv + j];
+          if (pij == 0.0 && sij == 0.0) continue;
+          for (long t = 0; t < D; ++t) {
+            dv[kv_index(d, b, j, g) + t] += pij * widen_bf16(dout[q_index(d, b, i, h) + t]);
+            dk[kv_index(d, b, j, g) + t] += scale * sij * widen_bf16(q[q_index(d, b, i, h) + t]);
+          }
+        }
+      for (long i = 0; i < Sq; ++i)
+        for (long t = 0; t < D; ++t) {
+          double acc = 0.0;
+          for (long j = 0; j < Skv; ++j)
+            acc += dS[i * Skv + j] * widen_bf16(k[kv_index(d, b, j, g) + t]);
+          dq[q_index(d, b, i, h) + t] = scale * acc;
+        }
     }
   }
   return 0;
