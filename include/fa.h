@@ -106,6 +106,28 @@ FA_API int fa_fwd_ext(const void* q, const void* k, const void* v, void* o, floa
                       int64_t mask_head_stride, void* stream);
 
 /*
+ * Backward pass: gradients of sum(dout * O) with respect to q, k, v for O = fa_fwd(q, k, v) with
+ * the same causal / window rule.  The probabilities are recomputed tile by tile from q, k and
+ * the forward pass's log-sum-exp rather than stored ("FlashAttention on Ascend NPUs",
+ * recomputation section).
+ *   q, o, dout  bf16 [B, Sq, Hq, D]      (o and lse as returned by fa_fwd for these inputs)
+ *   k, v        bf16 [B, Skv, Hkv, D]
+ *   lse         fp32 [B, Hq, Sq], natural log (required)
+ *   dq          bf16 [B, Sq, Hq, D]  written
+ *   dk, dv      bf16 [B, Skv, Hkv, D] written; for GQA / MQA they sum over the query heads that
+ *               read each KV head
+ *   workspace   at least fa_bwd_workspace_bytes(B, Hq, Sq) bytes (per-row D = dO . O and the
+ *               log-sum-exp in log2 units); contents on entry do not matter.
+ * Other arguments as for fa_fwd.  Three kernels run in order on `stream`; none uses atomics, so
+ * the result is deterministic.  Returns FA_OK or an fa_status error code.
+ */
+FA_API size_t fa_bwd_workspace_bytes(int B, int Hq, int Sq);
+FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq,
+                  int Skv, int D, float scale, int causal, int window, void* workspace,
+                  size_t workspace_bytes, void* stream);
+
+/*
  * Bytes of device workspace fa_decode_int8 needs: fp32 partial outputs [num_splits, B, Hq, D]
  * followed by fp32 partial log-sum-exps [num_splits, B, Hq], padded to 256 bytes.
  * Returns 0 for invalid sizes.

@@ -32,7 +32,8 @@ def test_header_declares_the_entry_points():
     names = declared_functions()
     for n in ("fa_fwd", "fa_decode_int8", "fa_decode_int8_workspace_bytes", "fa_status_string",
               "fa_device_status", "fa_selftest_bounded_wait", "fa_decode_int8_noalloc",
-              "fa_decode_int8_paged", "fa_decode_int4", "fa_decode_int4_paged", "fa_fwd_ext"):
+              "fa_decode_int8_paged", "fa_decode_int4", "fa_decode_int4_paged", "fa_fwd_ext", "fa_bwd",
+              "fa_bwd_workspace_bytes"):
         assert n in names
 
 
@@ -94,6 +95,31 @@ def test_fwd_ext_rejects(L, kw, code):
     assert L.fa_fwd_ext(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"],
                         a["Sq"], a["Skv"], a["D"], a["scale"], a["causal"], a["window"],
                         a["n_global"], a["mask"], a["sb"], a["sh"], None) == code
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(lse=None), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(dk=None), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(window=4), fa.STATUS["FA_ERR_INVALID_ARG"]),
+    (dict(D=80), fa.STATUS["FA_ERR_UNSUPPORTED"]),
+    (dict(dq=FAKE + 8), fa.STATUS["FA_ERR_ALIGNMENT"]),
+    (dict(ws_bytes=64), fa.STATUS["FA_ERR_WORKSPACE"]),
+])
+def test_bwd_rejects(L, kw, code):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, do=FAKE, lse=FAKE, dq=FAKE, dk=FAKE, dv=FAKE, B=1,
+             Hq=2, Hkv=2, Sq=128, Skv=128, D=64, scale=0.125, causal=0, window=0, ws=FAKE,
+             ws_bytes=None)
+    a.update(kw)
+    if a["ws_bytes"] is None:
+        a["ws_bytes"] = L.fa_bwd_workspace_bytes(a["B"], a["Hq"], a["Sq"])
+    assert L.fa_bwd(a["q"], a["k"], a["v"], a["o"], a["do"], a["lse"], a["dq"], a["dk"], a["dv"],
+                    a["B"], a["Hq"], a["Hkv"], a["Sq"], a["Skv"], a["D"], a["scale"], a["causal"],
+                    a["window"], a["ws"], a["ws_bytes"], None) == code
+
+
+def test_bwd_workspace_bytes(L):
+    assert fa.fa_bwd_workspace_bytes(2, 4, 300) == 2 * 2 * 4 * 384 * 4
+    assert fa.fa_bwd_workspace_bytes(0, 4, 300) == 0
 
 
 def dec(L, q=FAKE, k=FAKE, v=FAKE, ks=FAKE, vs=FAKE, o=FAKE, lse=None, B=2, Hq=8, Hkv=2, Skv=100,

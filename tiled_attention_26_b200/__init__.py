@@ -12,7 +12,7 @@ import ctypes
 import math
 import os
 
-__all__ = ["FaError", "lib", "fa_fwd", "fa_decode_int8", "fa_decode_int8_paged",
+__all__ = ["FaError", "lib", "fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_decode_int8", "fa_decode_int8_paged",
            "fa_decode_int4", "fa_decode_int4_paged", "fa_decode_int8_workspace_bytes",
            "fa_status_string", "fa_device_status", "fa_selftest_bounded_wait", "LIB_PATH",
            "STATUS"]
@@ -57,6 +57,10 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd_ext.argtypes = ([_P, _P, _P, _P, _P] + [_I] * 6 + [_F, _I, _I, _I, _P,
                                  ctypes.c_int64, ctypes.c_int64, _P])
         L.fa_fwd_ext.restype = _I
+        L.fa_bwd_workspace_bytes.argtypes = [_I, _I, _I]
+        L.fa_bwd_workspace_bytes.restype = _Z
+        L.fa_bwd.argtypes = [_P] * 9 + [_I] * 6 + [_F, _I, _I, _P, _Z, _P]
+        L.fa_bwd.restype = _I
         L.fa_decode_int8_workspace_bytes.argtypes = [_I, _I, _I, _I]
         L.fa_decode_int8_workspace_bytes.restype = _Z
         L.fa_decode_int8.argtypes = [_P] * 7 + [_I] * 5 + [_F, _I, _P, _Z, _P]
@@ -145,6 +149,45 @@ def fa_fwd(q, k, v, causal: bool = False, window: int = 0, scale: float | None =
     if rc != 0:
         raise FaError(rc, "fa_fwd")
     return o, lse
+
+
+def fa_bwd_workspace_bytes(B: int, Hq: int, Sq: int) -> int:
+    return int(lib().fa_bwd_workspace_bytes(int(B), int(Hq), int(Sq)))
+
+
+def fa_bwd(q, k, v, o, dout, lse, causal: bool = False, window: int = 0,
+           scale: float | None = None, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Backward pass of fa_fwd: gradients of sum(dout * o).  q, o, dout: bf16 [B, Sq, Hq, D];
+    k, v: bf16 [B, Skv, Hkv, D]; lse: fp32 [B, Hq, Sq] from fa_fwd.  Returns (dq, dk, dv)."""
+    import torch
+    B, Sq, Hq, D = q.shape
+    Skv, Hkv = k.shape[1], k.shape[2]
+    dev = q.device
+    _check(q, "q", torch.bfloat16, (B, Sq, Hq, D), dev)
+    _check(k, "k", torch.bfloat16, (B, Skv, Hkv, D), dev)
+    _check(v, "v", torch.bfloat16, (B, Skv, Hkv, D), dev)
+    _check(o, "o", torch.bfloat16, (B, Sq, Hq, D), dev)
+    _check(dout, "dout", torch.bfloat16, (B, Sq, Hq, D), dev)
+    _check(lse, "lse", torch.float32, (B, Hq, Sq), dev)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    _check(dq, "dq", torch.bfloat16, (B, Sq, Hq, D), dev)
+    _check(dk, "dk", torch.bfloat16, (B, Skv, Hkv, D), dev)
+    _check(dv, "dv", torch.bfloat16, (B, Skv, Hkv, D), dev)
+    need = fa_bwd_workspace_bytes(B, Hq, Sq)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(),
+                      lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, Hq, Hkv,
+                      Sq, Skv, D, float(scale), int(bool(causal)), int(window),
+                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                      _stream_ptr(stream))
+    if rc != 0:
+        raise FaError(rc, "fa_bwd")
+    return dq, dk, dv
 
 
 def fa_decode_int8_workspace_bytes(B: int, Hq: int, D: int, num_splits: int) -> int:

@@ -1,0 +1,614 @@
+// Attention backward pass for sm_100a.
+//
+// The forward pass keeps only O and the row log-sum-exp; the backward pass recomputes the
+// probabilities tile by tile instead of storing them ("FlashAttention on Ascend NPUs",
+// recomputation section).  With L the row log-sum-exp and D_i = dO_i . O_i:
+//   P_ij = exp(scale q_i.k_j - L_i),  dP_ij = dO_i . v_j,  dS_ij = P_ij (dP_ij - D_i)
+//   dV_j = sum_i P_ij dO_i,  dK_j = scale sum_i dS_ij q_i,  dQ_i = scale sum_j dS_ij k_j
+// Three kernels, none with atomics:
+//   fa_bwd_prep_kernel   D_i and L_i * log2(e) per (b, h, i) into a padded workspace
+//                        (padding rows get L = +inf, D = 0: they contribute nothing);
+//   fa_bwd_dkdv_kernel   one CTA per (b, KV head, 128-key tile): S^T = K Q^T and
+//                        dP^T = V dO^T per (query head of the group, 128-query tile), then
+//                        dV += P^T dO and dK += dS^T Q with P and dS in TMEM (GQA heads summed
+//                        in TMEM), one bf16 store of dK and dV at the end;
+//   fa_bwd_dq_kernel     one CTA per 128-row Q tile (query heads packed into rows as in the
+//                        forward pass): S = Q K^T and dP = dO V^T per key tile, then
+//                        dQ += dS K with dS in TMEM.
+// Warp roles (192 threads): warps 0-3 elementwise (thread = row = TMEM lane), warp 4 TMA
+// producer, warp 5 TMEM allocation + tcgen05.mma issue from one thread.
+#pragma once
+
+#include "prefill.cuh"
+#include "sm100.cuh"
+
+namespace fa {
+
+struct BwdParams {
+  int B, Hq, Hkv, Sq, Skv;
+  int G, Gp, NP;
+  int Sq_pad;          // rows of the per-(b, h) workspace vectors (multiple of 128)
+  int n_tiles;         // dQ: 128-row Q tiles per (b, KV head, head pack); dK/dV: key tiles
+  float scale;         // softmax scale
+  float scale_log2;    // scale * log2(e)
+  int causal, window;
+  const uint16_t* o;     // bf16 [B, Sq, Hq, D]
+  const uint16_t* dout;  // bf16 [B, Sq, Hq, D]
+  const float* lse;      // natural log [B, Hq, Sq]
+  float* lse2;           // workspace [B * Hq, Sq_pad]: L * log2(e)
+  float* delta;          // workspace [B * Hq, Sq_pad]: D
+  uint64_t timeout_ns;
+};
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kThreads = 192;
+  static constexpr int kHalves = D / 64;
+  static constexpr int kAtomBytes = 128 * 128;
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr uint32_t kTmemCols = 512;
+  // dQ kernel: Q and dO tiles, then a K/V ring
+  static constexpr int kQStages = (D == 128) ? 4 : 8;
+  static constexpr int kQOff = 0;
+  static constexpr int kDOOff = kTileBytes;
+  static constexpr int kQKVOff = 2 * kTileBytes;
+  static constexpr int kQBarOff = kQKVOff + kQStages * kTileBytes;
+  // barriers: in_full, kv_full[S], kv_empty[S], s_full, p_full, o_final, drain
+  static constexpr int kQNumBars = 5 + 2 * kQStages;
+  static constexpr int kQMiscOff = kQBarOff + 8 * kQNumBars;
+  static constexpr int kQSmemBytes = kQMiscOff + 16 + 1024;
+  // dK/dV kernel: K and V tiles, then a ring of (Q, dO, L, D) units
+  static constexpr int kUStages = (D == 128) ? 2 : 4;
+  static constexpr int kUnitBytes = 2 * kTileBytes + 2 * 128 * 4;
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = kTileBytes;
+  static constexpr int kUOff = 2 * kTileBytes;
+  static constexpr int kUBarOff = kUOff + kUStages * kUnitBytes;
+  // barriers: kv_full, u_full[S], u_empty[S], s_full, p_full, o_final, drain
+  static constexpr int kUNumBars = 5 + 2 * kUStages;
+  static constexpr int kUMiscOff = kUBarOff + 8 * kUNumBars;
+  static constexpr int kUSmemBytes = kUMiscOff + 16 + 1024;
+};
+
+// ---------------------------------------------------------------------------------------
+// D_i = dO_i . O_i and L_i * log2(e), one warp per (b, i, h) row; padding rows past Sq get
+// L = +inf and D = 0.  Rows with L = -inf (no visible key) also get +inf: their P is 0.
+// ---------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdParams p) {
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const long long rows = static_cast<long long>(p.B) * p.Hq * p.Sq_pad;
+  if (row >= rows) return;
+  const int i = static_cast<int>(row % p.Sq_pad);
+  const long long bh = row / p.Sq_pad;
+  const int h = static_cast<int>(bh % p.Hq), b = static_cast<int>(bh / p.Hq);
+  float acc = 0.f;
+  if (i < p.Sq) {
+    const size_t base = ((static_cast<size_t>(b) * p.Sq + i) * p.Hq + h) * D;
+#pragma unroll
+    for (int e = lane * 2; e < D; e += 64) {
+      const uint32_t o2 = *reinterpret_cast<const uint32_t*>(p.o + base + e);
+      const uint32_t d2 = *reinterpret_cast<const uint32_t*>(p.dout + base + e);
+      acc = fmaf(__uint_as_float(o2 << 16), __uint_as_float(d2 << 16), acc);
+      acc = fmaf(__uint_as_float(o2 & 0xFFFF0000u), __uint_as_float(d2 & 0xFFFF0000u), acc);
+    }
+  }
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  if (lane == 0) {
+    float l2 = INFINITY;
+    if (i < p.Sq) {
+      const float l = p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Sq + i];
+      l2 = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+    }
+    p.lse2[row] = l2;
+    p.delta[row] = (i < p.Sq) ? acc : 0.f;
+  }
+}
+
+// Query token i sees key k (bottom-right causal alignment, window of W keys).
+__device__ __forceinline__ bool bwd_visible(const BwdParams& p, int i, int k) {
+  const int ip = i + (p.Skv - p.Sq);
+  if (i >= p.Sq || k >= p.Skv) return false;
+  if (p.causal && k > ip) return false;
+  if (p.window > 0 && k <= ip - p.window) return false;
+  return true;
+}
+
+// ---------------------------------------------------------------------------------------
+// dK, dV: one CTA per (b, KV head g, key tile j).
+// ---------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
+                       const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ CUtensorMap tm_do,
+                       const __grid_constant__ CUtensorMap tm_vec,
+                       const __grid_constant__ CUtensorMap tm_dk,
+                       const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int idx) { return sb + C::kUBarOff + 8u * idx; };
+  constexpr int kBarKV = 0, kBarUFull = 1, kBarUEmpty = 1 + C::kUStages;
+  constexpr int kBarS = 1 + 2 * C::kUStages, kBarP = kBarS + 1, kBarO = kBarS + 2,
+                kBarDrain = kBarS + 3;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kUMiscOff);
+  int* abort_flag = reinterpret_cast<int*>(smem + C::kUMiscOff + 4);
+  const WaitCtl ctl{abort_flag, p.timeout_ns};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int j = static_cast<int>(blockIdx.x) % p.n_tiles;
+  const int bg = static_cast<int>(blockIdx.x) / p.n_tiles;
+  const int g = bg % p.Hkv, b = bg / p.Hkv;
+  const int k0 = 128 * j;
+  // query tiles whose rows see some key of [k0, k0 + 127]
+  const int off = p.Skv - p.Sq;
+  int i_lo = 0, i_hi = p.Sq - 1;
+  if (p.causal) i_lo = max(0, k0 - off);
+  if (p.window > 0) i_hi = min(p.Sq - 1, k0 + 127 + p.window - 1 - off);
+  const int qt_lo = i_lo / 128, qt_hi = (i_hi >= i_lo) ? i_hi / 128 : qt_lo - 1;
+  const int n_qt = max(0, qt_hi - qt_lo + 1);
+  const int n_units = n_qt * p.G;  // unit u: head g*G + u / n_qt, query tile qt_lo + u % n_qt
+
+  if (threadIdx.x == 0) {
+    for (int x = 0; x < C::kUNumBars; ++x)
+      mbar_init(bar(x), (x == kBarP) ? 128 : 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  constexpr uint32_t colS = 0, colDP = 128, colDV = 256, colDK = 256 + D;
+
+  if (warp == 4) {
+    // ============ producer ============
+    if (lane == 0 && n_units > 0) {
+      // (with no unit the epilogue writes zeros into these tiles: nothing may land there)
+      mbar_arrive_expect_tx(bar(kBarKV), 2 * C::kTileBytes);
+#pragma unroll
+      for (int hf = 0; hf < C::kHalves; ++hf) {
+        tma_load_4d(sb + C::kKOff + hf * C::kAtomBytes, &tm_k, bar(kBarKV), 64 * hf, g, k0, b);
+        tma_load_4d(sb + C::kVOff + hf * C::kAtomBytes, &tm_v, bar(kBarKV), 64 * hf, g, k0, b);
+      }
+      int issued = 0;
+      for (int u = 0; u < n_units; ++u) {
+        const int s = u % C::kUStages;
+        if (u >= C::kUStages &&
+            !mbar_wait(bar(kBarUEmpty + s), ((u / C::kUStages) - 1) & 1, ctl))
+          break;
+        const int h = g * p.G + u / n_qt, i0 = 128 * (qt_lo + u % n_qt);
+        const uint32_t base = sb + C::kUOff + s * C::kUnitBytes;
+        mbar_arrive_expect_tx(bar(kBarUFull + s), C::kUnitBytes);
+#pragma unroll
+        for (int hf = 0; hf < C::kHalves; ++hf) {
+          tma_load_4d(base + hf * C::kAtomBytes, &tm_q, bar(kBarUFull + s), 64 * hf, h, i0, b);
+          tma_load_4d(base + C::kTileBytes + hf * C::kAtomBytes, &tm_do, bar(kBarUFull + s),
+                      64 * hf, h, i0, b);
+        }
+        // L and D vectors: rows (b*Hq + h) of the two [B*Hq, Sq_pad] workspace arrays, which
+        // the vector map sees as one (Sq_pad, B*Hq, 2) tensor
+        const uint32_t vb = base + 2 * C::kTileBytes;
+        tma_load_3d(vb, &tm_vec, bar(kBarUFull + s), i0, b * p.Hq + h, 0);
+        tma_load_3d(vb + 512, &tm_vec, bar(kBarUFull + s), i0, b * p.Hq + h, 1);
+        issued = u + 1;
+      }
+      volatile int zero = 0;
+      const WaitCtl drain_ctl{&zero, p.timeout_ns};
+      mbar_wait(bar(kBarKV), 0, drain_ctl);
+      for (int s = 0; s < C::kUStages && s < issued; ++s) {
+        const int last = s + C::kUStages * ((issued - 1 - s) / C::kUStages);
+        mbar_wait(bar(kBarUFull + s), (last / C::kUStages) & 1, drain_ctl);
+      }
+    }
+  } else if (warp == 5) {
+    // ============ MMA issuer ============
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);
+      // D[tmem] = A_tile (K-major rows) . B_tile^T, K = D
+      auto mma_rows = [&](uint32_t d, uint32_t a, uint32_t bt) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t o2 = (kk / 4) * C::kAtomBytes + (kk % 4) * 32;
+          umma_ss(tmem + d, smem_desc_sw128(a + o2, 16, 1024), smem_desc_sw128(bt + o2, 16, 1024),
+                  idesc_s, kk > 0 ? 1u : 0u);
+        }
+      };
+      // D[tmem] (+)= A[tmem bf16, 128 x 128] . B_tile (MN-major, K = the tile's 128 rows)
+      auto mma_acc = [&](uint32_t d, uint32_t a_col, uint32_t bt, bool first) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tmem + d, tmem + a_col + kk * 8,
+                  smem_desc_sw128(bt + kk * 16 * 128, C::kAtomBytes, 1024), idesc_acc,
+                  (first && kk == 0) ? 0u : 1u);
+      };
+      bool ok = n_units > 0 && mbar_wait(bar(kBarKV), 0, ctl);
+      tc_fence_after();
+      for (int u = 0; u < n_units && ok; ++u) {
+        const int s = u % C::kUStages;
+        if (!(ok = mbar_wait(bar(kBarUFull + s), (u / C::kUStages) & 1, ctl))) break;
+        tc_fence_after();
+        const uint32_t qt = sb + C::kUOff + s * C::kUnitBytes, dot = qt + C::kTileBytes;
+        mma_rows(colS, sb + C::kKOff, qt);    // S^T = K Q^T
+        mma_rows(colDP, sb + C::kVOff, dot);  // dP^T = V dO^T
+        tc_commit(bar(kBarS));
+        if (!(ok = mbar_wait(bar(kBarP), u & 1, ctl))) break;
+        tc_fence_after();
+        mma_acc(colDV, colS, dot, u == 0);    // dV += P^T dO
+        mma_acc(colDK, colDP, qt, u == 0);    // dK += dS^T Q
+        tc_commit(bar(kBarUEmpty + s));
+      }
+      tc_commit(bar(kBarO));
+      tc_commit(bar(kBarDrain));
+      volatile int zero = 0;
+      const WaitCtl drain_ctl{&zero, p.timeout_ns};
+      mbar_wait(bar(kBarDrain), 0, drain_ctl);
+    }
+  } else {
+    // ============ elementwise: thread = key row ============
+    const int r = threadIdx.x;  // 0..127
+    const int key = k0 + r;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+    const float sl2 = p.scale_log2;
+    int n = 0;
+    for (int u = 0; u < n_units; ++u, ++n) {
+      const int s = u % C::kUStages;
+      bool ok = mbar_wait(bar(kBarS), u & 1, ctl);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const int i0 = 128 * (qt_lo + u % n_qt);
+      const float* vl = reinterpret_cast<const float*>(smem + C::kUOff + s * C::kUnitBytes +
+                                                       2 * C::kTileBytes);
+      const float* vd = vl + 128;
+      // every (query, key) of the tile visible?  (then no per-element test)
+      const bool full = bwd_visible(p, i0, k0 + 127) && bwd_visible(p, i0 + 127, k0) &&
+                        bwd_visible(p, i0, k0) && bwd_visible(p, i0 + 127, k0 + 127);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sv[2][32], dv[2][32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          tmem_ld32(trow + colS + 64 * half + 32 * c, sv[c]);
+          tmem_ld32(trow + colDP + 64 * half + 32 * c, dv[c]);
+        }
+        tmem_wait_ld();
+        uint32_t pp[32], ds[32];
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          float pv[2], dsv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int col = 2 * x + e;  // query column within this half
+            const int qc = 64 * half + col;
+            const float sval = __uint_as_float(sv[col / 32][col % 32]);
+            const float dpv = __uint_as_float(dv[col / 32][col % 32]);
+            float pr = ex2(fmaf(sval, sl2, -vl[qc]));
+            if (!full && !bwd_visible(p, i0 + qc, key)) pr = 0.f;
+            pv[e] = pr;
+            dsv[e] = pr * (dpv - vd[qc]);
+          }
+          pp[x] = pack_bf16x2(pv[0], pv[1]);
+          ds[x] = pack_bf16x2(dsv[0], dsv[1]);
+        }
+        tmem_st32(trow + colS + 32 * half, pp);
+        tmem_st32(trow + colDP + 32 * half, ds);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(kBarP));
+    }
+    // ---- epilogue: dV and scale * dK -> bf16 -> swizzled smem (the K / V tiles) -> TMA ----
+    bool have = false;
+    if (n_units > 0) {
+      bool ok = mbar_wait(bar(kBarO), 0, ctl);
+      have = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+    }
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      const uint32_t col = which ? colDK : colDV;
+      const float mul = which ? p.scale : 1.f;
+      uint8_t* stage = smem + (which ? C::kKOff : C::kVOff);
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t ov[32];
+        if (have) {
+          tmem_ld32(trow + col + 32 * c, ov);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int x = 0; x < 32; ++x) ov[x] = 0u;
+        }
+        const int hf = c >> 1;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(ov[8 * q4 + 0]) * mul, __uint_as_float(ov[8 * q4 + 1]) * mul);
+          w.y = pack_bf16x2(__uint_as_float(ov[8 * q4 + 2]) * mul, __uint_as_float(ov[8 * q4 + 3]) * mul);
+          w.z = pack_bf16x2(__uint_as_float(ov[8 * q4 + 4]) * mul, __uint_as_float(ov[8 * q4 + 5]) * mul);
+          w.w = pack_bf16x2(__uint_as_float(ov[8 * q4 + 6]) * mul, __uint_as_float(ov[8 * q4 + 7]) * mul);
+          const int chunk = ((c & 1) * 4 + q4) ^ (r & 7);
+          *reinterpret_cast<uint4*>(stage + hf * C::kAtomBytes + r * 128 + chunk * 16) = w;
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(1, 128);
+    if (r == 0) {
+#pragma unroll
+      for (int hf = 0; hf < C::kHalves; ++hf) {
+        tma_store_4d(&tm_dv, sb + C::kVOff + hf * C::kAtomBytes, 64 * hf, g, k0, b);
+        tma_store_4d(&tm_dk, sb + C::kKOff + hf * C::kAtomBytes, 64 * hf, g, k0, b);
+      }
+      tma_store_commit();
+      tma_store_wait_read_all();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// dQ: one CTA per 128-row Q tile; row r = (token t0 + r / Gp, head h0 + r % Gp).
+// ---------------------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
+                     const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v,
+                     const __grid_constant__ CUtensorMap tm_do,
+                     const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  auto bar = [&](int idx) { return sb + C::kQBarOff + 8u * idx; };
+  constexpr int kBarIn = 0, kBarKVFull = 1, kBarKVEmpty = 1 + C::kQStages;
+  constexpr int kBarS = 1 + 2 * C::kQStages, kBarP = kBarS + 1, kBarO = kBarS + 2,
+                kBarDrain = kBarS + 3;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kQMiscOff);
+  int* abort_flag = reinterpret_cast<int*>(smem + C::kQMiscOff + 4);
+  const WaitCtl ctl{abort_flag, p.timeout_ns};
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // heaviest (last) query tiles first
+  const int per_tile = p.B * p.Hkv * p.NP;
+  const int qt = p.n_tiles - 1 - static_cast<int>(blockIdx.x) / per_tile;
+  int rem = static_cast<int>(blockIdx.x) % per_tile;
+  const int b = rem / (p.Hkv * p.NP);
+  rem %= p.Hkv * p.NP;
+  const int g = rem / p.NP;
+  const int h0 = g * p.G + (rem % p.NP) * p.Gp;
+  const int tpt = 128 / p.Gp;
+  const int tok0 = qt * tpt;
+  // key tiles: the band of the tile's first and last tokens
+  const int first = tok0, last = min(tok0 + tpt, p.Sq) - 1;
+  const int off = p.Skv - p.Sq;
+  int jlo = 0, jhi = 0;
+  {
+    const int lo = p.window > 0 ? max(0, first + off - p.window + 1) : 0;
+    const int hi = p.causal ? min(last + off, p.Skv - 1) : p.Skv - 1;
+    if (hi >= lo && hi >= 0) {
+      jlo = lo / 128;
+      jhi = hi / 128 + 1;
+    }
+  }
+  const int n_kt = jhi - jlo;
+
+  if (threadIdx.x == 0) {
+    for (int x = 0; x < C::kQNumBars; ++x) mbar_init(bar(x), (x == kBarP) ? 128 : 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  constexpr uint32_t colS = 0, colDP = 128, colDQ = 256;
+
+  if (warp == 4) {
+    // ============ producer ============
+    if (lane == 0 && n_kt > 0) {
+      // (with no key tile the epilogue writes zeros into the Q tile: nothing may land there)
+      mbar_arrive_expect_tx(bar(kBarIn), 2 * C::kTileBytes);
+#pragma unroll
+      for (int hf = 0; hf < C::kHalves; ++hf) {
+        tma_load_4d(sb + C::kQOff + hf * C::kAtomBytes, &tm_q, bar(kBarIn), 64 * hf, h0, tok0, b);
+        tma_load_4d(sb + C::kDOOff + hf * C::kAtomBytes, &tm_do, bar(kBarIn), 64 * hf, h0, tok0, b);
+      }
+      int issued = 0;
+      bool ok = true;
+      for (int t = 0; t < n_kt && ok; ++t) {
+#pragma unroll
+        for (int kind = 0; kind < 2; ++kind) {
+          const int pos = 2 * t + kind;
+          const int s = pos % C::kQStages;
+          if (!mbar_wait(bar(kBarKVEmpty + s), ((pos / C::kQStages) & 1) ^ 1, ctl)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(bar(kBarKVFull + s), C::kTileBytes);
+#pragma unroll
+          for (int hf = 0; hf < C::kHalves; ++hf)
+            tma_load_4d(sb + C::kQKVOff + s * C::kTileBytes + hf * C::kAtomBytes,
+                        kind ? &tm_v : &tm_k, bar(kBarKVFull + s), 64 * hf, g, 128 * (jlo + t), b);
+          issued = pos + 1;
+        }
+      }
+      volatile int zero = 0;
+      const WaitCtl drain_ctl{&zero, p.timeout_ns};
+      mbar_wait(bar(kBarIn), 0, drain_ctl);
+      for (int s = 0; s < C::kQStages && s < issued; ++s) {
+        const int lastp = s + C::kQStages * ((issued - 1 - s) / C::kQStages);
+        mbar_wait(bar(kBarKVFull + s), (lastp / C::kQStages) & 1, drain_ctl);
+      }
+    }
+  } else if (warp == 5) {
+    // ============ MMA issuer ============
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
+      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);
+      auto mma_rows = [&](uint32_t d, uint32_t a, uint32_t bt) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t o2 = (kk / 4) * C::kAtomBytes + (kk % 4) * 32;
+          umma_ss(tmem + d, smem_desc_sw128(a + o2, 16, 1024), smem_desc_sw128(bt + o2, 16, 1024),
+                  idesc_s, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto kv_wait = [&](int pos) {
+        const bool r = mbar_wait(bar(kBarKVFull + pos % C::kQStages), (pos / C::kQStages) & 1, ctl);
+        tc_fence_after();
+        return r;
+      };
+      bool ok = n_kt > 0 && mbar_wait(bar(kBarIn), 0, ctl);
+      tc_fence_after();
+      for (int t = 0; t < n_kt && ok; ++t) {
+        const int kpos = 2 * t, vpos = kpos + 1;
+        const uint32_t kt = sb + C::kQKVOff + (kpos % C::kQStages) * C::kTileBytes;
+        const uint32_t vt = sb + C::kQKVOff + (vpos % C::kQStages) * C::kTileBytes;
+        if (!(ok = kv_wait(kpos))) break;
+        mma_rows(colS, sb + C::kQOff, kt);    // S = Q K^T
+        if (!(ok = kv_wait(vpos))) break;
+        mma_rows(colDP, sb + C::kDOOff, vt);  // dP = dO V^T
+        tc_commit(bar(kBarS));
+        tc_commit(bar(kBarKVEmpty + vpos % C::kQStages));
+        if (!(ok = mbar_wait(bar(kBarP), t & 1, ctl))) break;
+        tc_fence_after();
+        // dQ += dS K (K tile as the MN-major B operand)
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tmem + colDQ, tmem + colS + kk * 8,
+                  smem_desc_sw128(kt + kk * 16 * 128, C::kAtomBytes, 1024), idesc_acc,
+                  (t == 0 && kk == 0) ? 0u : 1u);
+        tc_commit(bar(kBarKVEmpty + kpos % C::kQStages));
+      }
+      tc_commit(bar(kBarO));
+      tc_commit(bar(kBarDrain));
+      volatile int zero = 0;
+      const WaitCtl drain_ctl{&zero, p.timeout_ns};
+      mbar_wait(bar(kBarDrain), 0, drain_ctl);
+    }
+  } else {
+    // ============ elementwise: thread = Q row ============
+    const int r = threadIdx.x;
+    const int i = tok0 + r / p.Gp;
+    const int hh = h0 + r % p.Gp;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+    const float sl2 = p.scale_log2;
+    const size_t vrow = (static_cast<size_t>(b) * p.Hq + hh) * p.Sq_pad + min(i, p.Sq_pad - 1);
+    const float l2 = p.lse2[vrow], dlt = p.delta[vrow];
+    const int ip = i + off;
+    const int my_lo = p.window > 0 ? max(0, ip - p.window + 1) : 0;
+    const int my_hi = p.causal ? min(ip, p.Skv - 1) : p.Skv - 1;
+    // rows of the tile that bound its masks (all rows of a tile share the key-tile range)
+    const int lo_last = p.window > 0 ? max(0, last + off - p.window + 1) : 0;
+    const int hi_first = p.causal ? min(first + off, p.Skv - 1) : p.Skv - 1;
+    for (int t = 0; t < n_kt; ++t) {
+      const int j = jlo + t;
+      bool ok = mbar_wait(bar(kBarS), t & 1, ctl);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      const bool need_mask = (128 * j < lo_last) || (128 * j + 127 > hi_first) || i >= p.Sq;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t sv[2][32], dv[2][32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          tmem_ld32(trow + colS + 64 * half + 32 * c, sv[c]);
+          tmem_ld32(trow + colDP + 64 * half + 32 * c, dv[c]);
+        }
+        tmem_wait_ld();
+        uint32_t ds[32];
+#pragma unroll
+        for (int x = 0; x < 32; ++x) {
+          float dsv[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int col = 2 * x + e;
+            const int key = 128 * j + 64 * half + col;
+            float pr = ex2(fmaf(__uint_as_float(sv[col / 32][col % 32]), sl2, -l2));
+            if (need_mask && (key < my_lo || key > my_hi || i >= p.Sq)) pr = 0.f;
+            dsv[e] = pr * (__uint_as_float(dv[col / 32][col % 32]) - dlt);
+          }
+          ds[x] = pack_bf16x2(dsv[0], dsv[1]);
+        }
+        tmem_st32(trow + colS + 32 * half, ds);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(kBarP));
+    }
+    // ---- epilogue: scale * dQ -> bf16 -> swizzled smem (the Q tile) -> TMA ----
+    bool have = false;
+    if (n_kt > 0) {
+      bool ok = mbar_wait(bar(kBarO), 0, ctl);
+      have = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+    }
+    uint8_t* stage = smem + C::kQOff;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t ov[32];
+      if (have) {
+        tmem_ld32(trow + colDQ + 32 * c, ov);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int x = 0; x < 32; ++x) ov[x] = 0u;
+      }
+      const int hf = c >> 1;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(ov[8 * q4 + 0]) * p.scale, __uint_as_float(ov[8 * q4 + 1]) * p.scale);
+        w.y = pack_bf16x2(__uint_as_float(ov[8 * q4 + 2]) * p.scale, __uint_as_float(ov[8 * q4 + 3]) * p.scale);
+        w.z = pack_bf16x2(__uint_as_float(ov[8 * q4 + 4]) * p.scale, __uint_as_float(ov[8 * q4 + 5]) * p.scale);
+        w.w = pack_bf16x2(__uint_as_float(ov[8 * q4 + 6]) * p.scale, __uint_as_float(ov[8 * q4 + 7]) * p.scale);
+        const int chunk = ((c & 1) * 4 + q4) ^ (r & 7);
+        *reinterpret_cast<uint4*>(stage + hf * C::kAtomBytes + r * 128 + chunk * 16) = w;
+      }
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(1, 128);
+    if (r == 0 && tok0 < p.Sq) {
+#pragma unroll
+      for (int hf = 0; hf < C::kHalves; ++hf)
+        tma_store_4d(&tm_dq, sb + C::kQOff + hf * C::kAtomBytes, 64 * hf, h0, tok0, b);
+      tma_store_commit();
+      tma_store_wait_read_all();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace fa

@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "../../include/fa.h"
+#include "backward.cuh"
 #include "decode.cuh"
 #include "prefill.cuh"
 #include "sm100.cuh"
@@ -156,6 +157,101 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
   }
   if (regs < C::kMinLaunchRegs) return FA_ERR_UNSUPPORTED;
   kernel<<<static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// fp32 [n2][n1][n0] array as a 3-D tensor; a box is `box0` consecutive elements of one row.
+int encode_f32_3d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1, uint64_t n2,
+                  uint32_t box0) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return FA_ERR_CUDA;
+  const cuuint64_t dims[3] = {n0, n1, n2};
+  const cuuint64_t strides[2] = {n0 * 4, n0 * n1 * 4};
+  const cuuint32_t box[3] = {box0, 1, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+int bwd_sq_pad(int Sq) { return (Sq + 127) / 128 * 128; }
+
+size_t bwd_ws_bytes(int B, int Hq, int Sq) {
+  return 2ull * static_cast<size_t>(B) * Hq * bwd_sq_pad(Sq) * sizeof(float);
+}
+
+std::atomic<uint64_t> g_attr_bwd[4];
+
+template <int D>
+int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+               const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq,
+               int Skv, float scale, int causal, int window, void* ws, cudaStream_t stream) {
+  using C = fa::BwdCfg<D>;
+  fa::BwdParams p{};
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Sq = Sq;
+  p.Skv = Skv;
+  p.G = Hq / Hkv;
+  p.Gp = 1;
+  while (p.Gp < 8 && p.G % (2 * p.Gp) == 0) p.Gp *= 2;
+  p.NP = p.G / p.Gp;
+  p.Sq_pad = bwd_sq_pad(Sq);
+  p.scale = scale;
+  p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  p.causal = causal;
+  p.window = window;
+  p.o = static_cast<const uint16_t*>(o);
+  p.dout = static_cast<const uint16_t*>(dout);
+  p.lse = lse;
+  p.lse2 = static_cast<float*>(ws);
+  p.delta = p.lse2 + static_cast<size_t>(B) * Hq * p.Sq_pad;
+  p.timeout_ns = kKernelTimeoutNs;
+
+  // 1. D and L * log2(e)
+  const long long rows = static_cast<long long>(B) * Hq * p.Sq_pad;
+  if ((rows + 7) / 8 > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  fa::fa_bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+
+  int rc;
+  CUtensorMap tk, tv, tq1, tdo1, tvec, tdk, tdv;
+  if ((rc = encode_bf16_4d(&tk, k, D, Hkv, Skv, B, 1, 128)) != FA_OK) return rc;
+  if ((rc = encode_bf16_4d(&tv, v, D, Hkv, Skv, B, 1, 128)) != FA_OK) return rc;
+  if ((rc = encode_bf16_4d(&tq1, q, D, Hq, Sq, B, 1, 128)) != FA_OK) return rc;
+  if ((rc = encode_bf16_4d(&tdo1, dout, D, Hq, Sq, B, 1, 128)) != FA_OK) return rc;
+  if ((rc = encode_f32_3d(&tvec, ws, p.Sq_pad, static_cast<uint64_t>(B) * Hq, 2, 128)) != FA_OK)
+    return rc;
+  if ((rc = encode_bf16_4d(&tdk, dk, D, Hkv, Skv, B, 1, 128)) != FA_OK) return rc;
+  if ((rc = encode_bf16_4d(&tdv, dv, D, Hkv, Skv, B, 1, 128)) != FA_OK) return rc;
+
+  // 2. dK, dV: one CTA per (b, KV head, key tile)
+  p.n_tiles = (Skv + 127) / 128;
+  const long long grid_kv = static_cast<long long>(p.n_tiles) * B * Hkv;
+  if (grid_kv > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  auto kdkdv = fa::fa_bwd_dkdv_kernel<D>;
+  if ((rc = ensure_smem_attr(kdkdv, C::kUSmemBytes, g_attr_bwd[D == 128 ? 0 : 1])) != FA_OK)
+    return rc;
+  kdkdv<<<static_cast<unsigned>(grid_kv), C::kThreads, C::kUSmemBytes, stream>>>(
+      tq1, tk, tv, tdo1, tvec, tdk, tdv, p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+
+  // 3. dQ: one CTA per 128-row Q tile (query heads packed into rows as in the forward pass)
+  const uint32_t tpt = 128 / p.Gp;
+  CUtensorMap tq, tdo, tdq;
+  if ((rc = encode_bf16_4d(&tq, q, D, Hq, Sq, B, p.Gp, tpt)) != FA_OK) return rc;
+  if ((rc = encode_bf16_4d(&tdo, dout, D, Hq, Sq, B, p.Gp, tpt)) != FA_OK) return rc;
+  if ((rc = encode_bf16_4d(&tdq, dq, D, Hq, Sq, B, p.Gp, tpt)) != FA_OK) return rc;
+  p.n_tiles = (Sq + static_cast<int>(tpt) - 1) / static_cast<int>(tpt);
+  const long long grid_q = static_cast<long long>(p.n_tiles) * B * Hkv * p.NP;
+  if (grid_q > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  auto kdq = fa::fa_bwd_dq_kernel<D>;
+  if ((rc = ensure_smem_attr(kdq, C::kQSmemBytes, g_attr_bwd[D == 128 ? 2 : 3])) != FA_OK)
+    return rc;
+  kdq<<<static_cast<unsigned>(grid_q), C::kThreads, C::kQSmemBytes, stream>>>(tq, tk, tv, tdo,
+                                                                              tdq, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -417,6 +513,35 @@ int fa_fwd_ext(const void* q, const void* k, const void* v, void* o, float* lse,
   FA_PREFILL_CASE(64, 3)
 #undef FA_PREFILL_CASE
   return FA_ERR_UNSUPPORTED;
+}
+
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Sq) {
+  if (B <= 0 || Hq <= 0 || Sq <= 0) return 0;
+  return bwd_ws_bytes(B, Hq, Sq);
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+           const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Sq,
+           int Skv, int D, float scale, int causal, int window, void* workspace,
+           size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Sq <= 0 || Skv <= 0 || D <= 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (window < 0 || (window > 0 && !causal)) return FA_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return FA_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+      (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return FA_ERR_ALIGNMENT;
+  if (!workspace || workspace_bytes < bwd_ws_bytes(B, Hq, Sq)) return FA_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return FA_ERR_ALIGNMENT;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return D == 128 ? launch_bwd<128>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Sq, Skv, scale,
+                                    causal, window, workspace, s)
+                  : launch_bwd<64>(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Sq, Skv, scale,
+                                   causal, window, workspace, s);
 }
 
 size_t fa_decode_int8_workspace_bytes(int B, int Hq, int D, int num_splits) {
