@@ -156,6 +156,24 @@ def measure_mask_variants(fa, synthetic, torch, dev, stream, steps: int, warmup:
     return out
 
 
+def measure_backward(fa, synthetic, torch, dev, stream, steps: int, warmup: int):
+    """fa_bwd on the MHA causal workload (its own loop; the forward pass runs once, outside the
+    timing).  Returns (ms per call, algorithmic flops = 10*D per visible pair: the five products
+    S, dP, dV, dK, dQ)."""
+    w = synthetic.WORKLOADS["mha_causal"]
+    q, k, v = synthetic.make_qkv_torch(w, dev)
+    do = synthetic.normal_bf16_torch(w.seed(3), w.q_shape(), dev)
+    o, lse = fa.fa_fwd(q, k, v, causal=True, scale=w.scale, stream=stream)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.fa_bwd_workspace_bytes(w.B, w.Hq, w.Sq), dtype=torch.uint8, device=dev)
+    ms = time_calls(torch, stream,
+                    lambda: fa.fa_bwd(q, k, v, o, do, lse, causal=True, scale=w.scale, dq=dq,
+                                      dk=dk, dv=dv, workspace=ws, stream=stream), steps, warmup)
+    if fa.fa_device_status() != 0:
+        raise RuntimeError("the backward pass reported a device-side error")
+    return ms, prefill_flops(w) // 4 * 10
+
+
 def measure_paged_decode(fa, synthetic, torch, dev, stream, steps: int, warmup: int):
     """Time fa_decode_int8_paged on the paged workload (its own short loop after the step loop).
     Returns (ms per call averaged over ``steps`` launches, algorithmic bytes per call)."""
@@ -478,6 +496,9 @@ def main():
     mv = measure_mask_variants(fa, synthetic, torch, dev, stream, steps=min(K, 100),
                                warmup=max(3, args.warmup // 4))
     mv = {kk: (max_over_ranks(ms), fl) for kk, (ms, fl) in mv.items()}
+    bw_ms, bw_flops = measure_backward(fa, synthetic, torch, dev, stream, steps=min(K, 50),
+                                       warmup=max(3, args.warmup // 4))
+    bw_ms = max_over_ranks(bw_ms)
 
     # ---- end to end through the public API, host buffers, copies inside the timed region ----
     e2e = None
@@ -596,6 +617,12 @@ def main():
                 "unit": "TFLOP/s",
                 "frac": mv["global_local"][1] / (mv["global_local"][0] * 1e-3) / 1e12
                         / peaks["bf16_tflops_sustained"]},
+            "backward": {
+                "workload": "mha_causal (B=2, H=32, S=4096, D=128, causal): fa_bwd after fa_fwd",
+                "kernels": "fa_bwd_prep_kernel + fa_bwd_dkdv_kernel<128> + fa_bwd_dq_kernel<128>",
+                "ms_per_call": bw_ms, "flops_per_call": bw_flops,
+                "achieved": bw_flops / (bw_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "frac": bw_flops / (bw_ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 3 * K,

@@ -92,3 +92,24 @@ def test_backward_invariants(fa):
     dof = synthetic.bf16_bits_to_f32(do).astype(np.float64)
     np.testing.assert_allclose(dv.sum(axis=1), dof.sum(axis=1), atol=0.05 * np.abs(dof.sum(axis=1)).max())
     assert np.abs(dk.sum(axis=1)).max() <= 0.02 * np.abs(dk).max() * math.sqrt(S)
+
+
+def test_backward_full_size_one_head(fa):
+    # the MHA causal workload (B=2, H=32, S=4096, D=128) through the kernels; the oracle checks
+    # head (b=1, h=31) in full (an MHA head's gradients depend on that head's inputs only)
+    import torch
+    w = synthetic.WORKLOADS["mha_causal"]
+    q, k, v = synthetic.make_qkv_torch(w, "cuda")
+    do = synthetic.normal_bf16_torch(w.seed(3), w.q_shape(), "cuda")
+    o, lse = fa.fa_fwd(q, k, v, causal=True, scale=w.scale)
+    dq, dk, dv = fa.fa_bwd(q, k, v, o, do, lse, causal=True, scale=w.scale)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status() == 0
+    from parity_util import to_host_bits
+    b, h = 1, 31
+    sl = lambda t: np.ascontiguousarray(to_host_bits(t[b:b + 1, :, h:h + 1]))
+    rq, rk, rv = oracle.attn_bwd(sl(q), sl(k), sl(v), sl(do), w.scale, 1, 0)
+    g = lambda t: t[b:b + 1, :, h:h + 1].float().cpu().numpy().astype(np.float64)
+    _check("dq", g(dq), rq, "mha_causal full b1 h31")
+    _check("dk", g(dk), rk, "mha_causal full b1 h31")
+    _check("dv", g(dv), rv, "mha_causal full b1 h31")
