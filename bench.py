@@ -370,6 +370,28 @@ def run_reference(args):
     return 0
 
 
+def run_only_backward(args):
+    """fa_bwd on the MHA causal workload alone, one JSON line (used to profile the backward
+    kernels without the other workloads resident on the device)."""
+    import torch
+
+    import synthetic
+    import tiled_attention_26_b200 as fa
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    ms, flops = measure_backward(fa, synthetic, torch, dev, stream, steps=args.steps,
+                                 warmup=args.warmup)
+    peaks, _ = load_peaks()
+    print(json.dumps({"metric": "attention backward TFLOP/s (10*D flops per visible pair)",
+                      "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                      "ms_per_call": ms, "steps": args.steps, "warmup": args.warmup,
+                      "frac": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"],
+                      "config": {"workload": "mha_causal (B=2, H=32, S=4096, D=128, causal)"}}),
+          flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -379,9 +401,13 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["backward"], default=None,
+                    help="time one further row on its own (for profiling); prints its own line")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.only == "backward":
+        return run_only_backward(args)
 
     import torch
 

@@ -6,7 +6,7 @@
 //   P_ij = exp(scale q_i.k_j - L_i),  dP_ij = dO_i . v_j,  dS_ij = P_ij (dP_ij - D_i)
 //   dV_j = sum_i P_ij dO_i,  dK_j = scale sum_i dS_ij q_i,  dQ_i = scale sum_j dS_ij k_j
 // Three kernels, none with atomics:
-//   fa_bwd_prep_kernel   D_i and L_i * log2(e) per (b, h, i) into a padded workspace
+//   fa_bwd_prep_kernel   -D_i and -L_i * log2(e) per (b, h, i) into a padded workspace
 //                        (padding rows get L = +inf, D = 0: they contribute nothing);
 //   fa_bwd_dkdv_kernel   one CTA per (b, KV head, 128-key tile): S^T = K Q^T and
 //                        dP^T = V dO^T per (query head of the group, 128-query tile), then
@@ -15,8 +15,9 @@
 //   fa_bwd_dq_kernel     one CTA per 128-row Q tile (query heads packed into rows as in the
 //                        forward pass): S = Q K^T and dP = dO V^T per key tile, then
 //                        dQ += dS K with dS in TMEM.
-// Warp roles (192 threads): warps 0-3 elementwise (thread = row = TMEM lane), warp 4 TMA
-// producer, warp 5 TMEM allocation + tcgen05.mma issue from one thread.
+// Warp roles (320 threads): warps 0-7 elementwise (thread = row = TMEM lane of its quadrant;
+// warps w and w + 4 share a quadrant and take one half of the columns each), warp 8 TMA
+// producer, warp 9 TMEM allocation + tcgen05.mma issue from one thread.
 #pragma once
 
 #include "prefill.cuh"
@@ -35,14 +36,14 @@ struct BwdParams {
   const uint16_t* o;     // bf16 [B, Sq, Hq, D]
   const uint16_t* dout;  // bf16 [B, Sq, Hq, D]
   const float* lse;      // natural log [B, Hq, Sq]
-  float* lse2;           // workspace [B * Hq, Sq_pad]: L * log2(e)
-  float* delta;          // workspace [B * Hq, Sq_pad]: D
+  float* lse2;           // workspace [B * Hq, Sq_pad]: -L * log2(e)
+  float* delta;          // workspace [B * Hq, Sq_pad]: -D
   uint64_t timeout_ns;
 };
 
 template <int D>
 struct BwdCfg {
-  static constexpr int kThreads = 192;
+  static constexpr int kThreads = 320;
   static constexpr int kHalves = D / 64;
   static constexpr int kAtomBytes = 128 * 128;
   static constexpr int kTileBytes = 128 * D * 2;
@@ -53,8 +54,9 @@ struct BwdCfg {
   static constexpr int kDOOff = kTileBytes;
   static constexpr int kQKVOff = 2 * kTileBytes;
   static constexpr int kQBarOff = kQKVOff + kQStages * kTileBytes;
-  // barriers: in_full, kv_full[S], kv_empty[S], s_full, p_full, o_final, drain
-  static constexpr int kQNumBars = 5 + 2 * kQStages;
+  // barriers: in_full, kv_full[S], kv_empty[S], sdp_full, sdp_free, ds_ready, dq_done,
+  // o_final, drain
+  static constexpr int kQNumBars = 7 + 2 * kQStages;
   static constexpr int kQMiscOff = kQBarOff + 8 * kQNumBars;
   static constexpr int kQSmemBytes = kQMiscOff + 16 + 1024;
   // dK/dV kernel: K and V tiles, then a ring of (Q, dO, L, D) units
@@ -64,15 +66,17 @@ struct BwdCfg {
   static constexpr int kVOff = kTileBytes;
   static constexpr int kUOff = 2 * kTileBytes;
   static constexpr int kUBarOff = kUOff + kUStages * kUnitBytes;
-  // barriers: kv_full, u_full[S], u_empty[S], s_full, p_full, o_final, drain
-  static constexpr int kUNumBars = 5 + 2 * kUStages;
+  // barriers: kv_full, u_full[S], u_empty[S], s_full, dp_full, p_ready, ds_ready, o_final,
+  // drain
+  static constexpr int kUNumBars = 7 + 2 * kUStages;
   static constexpr int kUMiscOff = kUBarOff + 8 * kUNumBars;
   static constexpr int kUSmemBytes = kUMiscOff + 16 + 1024;
 };
 
 // ---------------------------------------------------------------------------------------
-// D_i = dO_i . O_i and L_i * log2(e), one warp per (b, i, h) row; padding rows past Sq get
-// L = +inf and D = 0.  Rows with L = -inf (no visible key) also get +inf: their P is 0.
+// -D_i = -dO_i . O_i and -L_i * log2(e), one warp per (b, i, h) row (stored negated so the
+// kernels add them); padding rows past Sq get L = +inf and D = 0.  Rows with L = -inf (no
+// visible key) also get +inf: their P is 0.
 // ---------------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdParams p) {
@@ -102,8 +106,8 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdParams p) {
       const float l = p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Sq + i];
       l2 = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
     }
-    p.lse2[row] = l2;
-    p.delta[row] = (i < p.Sq) ? acc : 0.f;
+    p.lse2[row] = -l2;
+    p.delta[row] = (i < p.Sq) ? -acc : 0.f;
   }
 }
 
@@ -120,7 +124,7 @@ __device__ __forceinline__ bool bwd_visible(const BwdParams& p, int i, int k) {
 // dK, dV: one CTA per (b, KV head g, key tile j).
 // ---------------------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                        const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_v,
@@ -135,8 +139,8 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t sb = smem_u32(smem);
   auto bar = [&](int idx) { return sb + C::kUBarOff + 8u * idx; };
   constexpr int kBarKV = 0, kBarUFull = 1, kBarUEmpty = 1 + C::kUStages;
-  constexpr int kBarS = 1 + 2 * C::kUStages, kBarP = kBarS + 1, kBarO = kBarS + 2,
-                kBarDrain = kBarS + 3;
+  constexpr int kBarS = 1 + 2 * C::kUStages, kBarDP = kBarS + 1, kBarP = kBarS + 2,
+                kBarDS = kBarS + 3, kBarO = kBarS + 4, kBarDrain = kBarS + 5;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kUMiscOff);
   int* abort_flag = reinterpret_cast<int*>(smem + C::kUMiscOff + 4);
   const WaitCtl ctl{abort_flag, p.timeout_ns};
@@ -157,11 +161,11 @@ __global__ void __launch_bounds__(192, 1)
 
   if (threadIdx.x == 0) {
     for (int x = 0; x < C::kUNumBars; ++x)
-      mbar_init(bar(x), (x == kBarP) ? 128 : 1);
+      mbar_init(bar(x), (x == kBarP || x == kBarDS) ? 256 : 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
     tmem_relinquish();
   }
@@ -171,7 +175,7 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = *tmem_holder;
   constexpr uint32_t colS = 0, colDP = 128, colDV = 256, colDK = 256 + D;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ============ producer ============
     if (lane == 0 && n_units > 0) {
       // (with no unit the epilogue writes zeros into these tiles: nothing may land there)
@@ -211,7 +215,7 @@ __global__ void __launch_bounds__(192, 1)
         mbar_wait(bar(kBarUFull + s), (last / C::kUStages) & 1, drain_ctl);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ============ MMA issuer ============
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
@@ -225,29 +229,56 @@ __global__ void __launch_bounds__(192, 1)
                   idesc_s, kk > 0 ? 1u : 0u);
         }
       };
-      // D[tmem] (+)= A[tmem bf16, 128 x 128] . B_tile (MN-major, K = the tile's 128 rows)
+      // D[tmem] (+)= A[tmem bf16, 128 x 128] . B_tile (MN-major, K = the tile's 128 rows);
+      // A's queries 0-63 sit in columns [a_col, a_col + 32), queries 64-127 in
+      // [a_col + 64, a_col + 96)
       auto mma_acc = [&](uint32_t d, uint32_t a_col, uint32_t bt, bool first) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tmem + d, tmem + a_col + kk * 8,
+          umma_ts(tmem + d, tmem + a_col + 64 * (kk / 4) + 8 * (kk % 4),
                   smem_desc_sw128(bt + kk * 16 * 128, C::kAtomBytes, 1024), idesc_acc,
                   (first && kk == 0) ? 0u : 1u);
       };
+      // Order: S(0) dP(0) | dV(u) S(u+1) | dK(u) dP(u+1) | ...: the tensor core works on the
+      // next unit's products while the elementwise warps turn S into P and dP into dS.
+      auto unit_tiles = [&](int u, uint32_t& qt, uint32_t& dot) {
+        qt = sb + C::kUOff + (u % C::kUStages) * C::kUnitBytes;
+        dot = qt + C::kTileBytes;
+      };
       bool ok = n_units > 0 && mbar_wait(bar(kBarKV), 0, ctl);
       tc_fence_after();
-      for (int u = 0; u < n_units && ok; ++u) {
-        const int s = u % C::kUStages;
-        if (!(ok = mbar_wait(bar(kBarUFull + s), (u / C::kUStages) & 1, ctl))) break;
+      if (ok && (ok = mbar_wait(bar(kBarUFull), 0, ctl))) {
         tc_fence_after();
-        const uint32_t qt = sb + C::kUOff + s * C::kUnitBytes, dot = qt + C::kTileBytes;
+        uint32_t qt, dot;
+        unit_tiles(0, qt, dot);
         mma_rows(colS, sb + C::kKOff, qt);    // S^T = K Q^T
-        mma_rows(colDP, sb + C::kVOff, dot);  // dP^T = V dO^T
         tc_commit(bar(kBarS));
+        mma_rows(colDP, sb + C::kVOff, dot);  // dP^T = V dO^T
+        tc_commit(bar(kBarDP));
+      }
+      for (int u = 0; u < n_units && ok; ++u) {
+        uint32_t qt, dot, qn = 0, don = 0;
+        unit_tiles(u, qt, dot);
+        const bool nxt = u + 1 < n_units;
         if (!(ok = mbar_wait(bar(kBarP), u & 1, ctl))) break;
         tc_fence_after();
         mma_acc(colDV, colS, dot, u == 0);    // dV += P^T dO
+        if (nxt) {
+          if (!(ok = mbar_wait(bar(kBarUFull + (u + 1) % C::kUStages), ((u + 1) / C::kUStages) & 1, ctl)))
+            break;
+          tc_fence_after();
+          unit_tiles(u + 1, qn, don);
+          mma_rows(colS, sb + C::kKOff, qn);  // S^T of the next unit (after dV read P)
+          tc_commit(bar(kBarS));
+        }
+        if (!(ok = mbar_wait(bar(kBarDS), u & 1, ctl))) break;
+        tc_fence_after();
         mma_acc(colDK, colDP, qt, u == 0);    // dK += dS^T Q
-        tc_commit(bar(kBarUEmpty + s));
+        tc_commit(bar(kBarUEmpty + u % C::kUStages));
+        if (nxt) {
+          mma_rows(colDP, sb + C::kVOff, don);  // dP^T of the next unit (after dK read dS)
+          tc_commit(bar(kBarDP));
+        }
       }
       tc_commit(bar(kBarO));
       tc_commit(bar(kBarDrain));
@@ -256,70 +287,98 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(bar(kBarDrain), 0, drain_ctl);
     }
   } else {
-    // ============ elementwise: thread = key row ============
-    const int r = threadIdx.x;  // 0..127
+    // ============ elementwise: thread = key row; this warp's half of the query columns ====
+    const int wq = warp & 3, ch = warp >> 2;
+    const int r = 32 * wq + lane;
     const int key = k0 + r;
-    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * warp) << 16);
-    const float sl2 = p.scale_log2;
-    int n = 0;
-    for (int u = 0; u < n_units; ++u, ++n) {
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * wq) << 16);
+    const uint64_t sl2 = f2(p.scale_log2, p.scale_log2);
+    for (int u = 0; u < n_units; ++u) {
       const int s = u % C::kUStages;
+      const int i0 = 128 * (qt_lo + u % n_qt);
+      // -L log2(e) and -D of the unit's 128 queries (broadcast reads, four at a time)
+      const float4* vl = reinterpret_cast<const float4*>(smem + C::kUOff + s * C::kUnitBytes +
+                                                         2 * C::kTileBytes) + 16 * ch;
+      const float4* vd = vl + 32;
+      // every (query, key) of the tile visible?  (then no per-element test)
+      const bool full = bwd_visible(p, i0, k0 + 127) && bwd_visible(p, i0 + 127, k0);
+      // ---- P = 2^(S^T scale log2 e - L) over this warp's 64 query columns, kept as bf16 ----
       bool ok = mbar_wait(bar(kBarS), u & 1, ctl);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      const int i0 = 128 * (qt_lo + u % n_qt);
-      const float* vl = reinterpret_cast<const float*>(smem + C::kUOff + s * C::kUnitBytes +
-                                                       2 * C::kTileBytes);
-      const float* vd = vl + 128;
-      // every (query, key) of the tile visible?  (then no per-element test)
-      const bool full = bwd_visible(p, i0, k0 + 127) && bwd_visible(p, i0 + 127, k0) &&
-                        bwd_visible(p, i0, k0) && bwd_visible(p, i0 + 127, k0 + 127);
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t sv[2][32], dv[2][32];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          tmem_ld32(trow + colS + 64 * half + 32 * c, sv[c]);
-          tmem_ld32(trow + colDP + 64 * half + 32 * c, dv[c]);
-        }
+      uint32_t pk[32];
+      {
+        uint32_t sv[64];
+        tmem_ld32(trow + colS + 64 * ch, *reinterpret_cast<uint32_t(*)[32]>(sv));
+        tmem_ld32(trow + colS + 64 * ch + 32, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
         tmem_wait_ld();
-        uint32_t pp[32], ds[32];
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          float pv[2], dsv[2];
+        for (int q = 0; q < 16; ++q) {
+          const float4 nl = vl[q];
+          float x0, x1, x2, x3;
+          f2_split(f2_fma(f2(__uint_as_float(sv[4 * q]), __uint_as_float(sv[4 * q + 1])), sl2,
+                          f2(nl.x, nl.y)), x0, x1);
+          f2_split(f2_fma(f2(__uint_as_float(sv[4 * q + 2]), __uint_as_float(sv[4 * q + 3])), sl2,
+                          f2(nl.z, nl.w)), x2, x3);
+          float e[4] = {ex2(x0), ex2(x1), ex2(x2), ex2(x3)};
+          if (!full) {
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = 2 * x + e;  // query column within this half
-            const int qc = 64 * half + col;
-            const float sval = __uint_as_float(sv[col / 32][col % 32]);
-            const float dpv = __uint_as_float(dv[col / 32][col % 32]);
-            float pr = ex2(fmaf(sval, sl2, -vl[qc]));
-            if (!full && !bwd_visible(p, i0 + qc, key)) pr = 0.f;
-            pv[e] = pr;
-            dsv[e] = pr * (dpv - vd[qc]);
+            for (int t = 0; t < 4; ++t)
+              if (!bwd_visible(p, i0 + 64 * ch + 4 * q + t, key)) e[t] = 0.f;
           }
-          pp[x] = pack_bf16x2(pv[0], pv[1]);
-          ds[x] = pack_bf16x2(dsv[0], dsv[1]);
+          pk[2 * q] = pack_bf16x2(e[0], e[1]);
+          pk[2 * q + 1] = pack_bf16x2(e[2], e[3]);
         }
-        tmem_st32(trow + colS + 32 * half, pp);
-        tmem_st32(trow + colDP + 32 * half, ds);
       }
+      // each warp writes its 64 queries' P (32 bf16 pairs) over the first half of the S^T
+      // columns it read itself, so the two warps of a quadrant never touch each other's input
+      tmem_st32(trow + colS + 64 * ch, pk);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(kBarP));
+      // ---- dS = P (dP^T - D) ----
+      ok = mbar_wait(bar(kBarDP), u & 1, ctl);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      {
+        uint32_t dv[64];
+        tmem_ld32(trow + colDP + 64 * ch, *reinterpret_cast<uint32_t(*)[32]>(dv));
+        tmem_ld32(trow + colDP + 64 * ch + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
+        tmem_wait_ld();
+        uint32_t ds[32];
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const float4 nd = vd[q];
+          const uint64_t p01 = f2(__uint_as_float(pk[2 * q] << 16),
+                                  __uint_as_float(pk[2 * q] & 0xFFFF0000u));
+          const uint64_t p23 = f2(__uint_as_float(pk[2 * q + 1] << 16),
+                                  __uint_as_float(pk[2 * q + 1] & 0xFFFF0000u));
+          float d0, d1, d2, d3;
+          f2_split(f2_mul(p01, f2_add(f2(__uint_as_float(dv[4 * q]), __uint_as_float(dv[4 * q + 1])),
+                                      f2(nd.x, nd.y))), d0, d1);
+          f2_split(f2_mul(p23, f2_add(f2(__uint_as_float(dv[4 * q + 2]), __uint_as_float(dv[4 * q + 3])),
+                                      f2(nd.z, nd.w))), d2, d3);
+          ds[2 * q] = pack_bf16x2(d0, d1);
+          ds[2 * q + 1] = pack_bf16x2(d2, d3);
+        }
+        tmem_st32(trow + colDP + 64 * ch, ds);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(kBarDS));
     }
-    // ---- epilogue: dV and scale * dK -> bf16 -> swizzled smem (the K / V tiles) -> TMA ----
+    // ---- epilogue: warps 0-3 write dV, warps 4-7 scale * dK: bf16 -> swizzled smem (the
+    // V / K tiles) -> TMA ----
     bool have = false;
     if (n_units > 0) {
       bool ok = mbar_wait(bar(kBarO), 0, ctl);
       have = __all_sync(0xffffffffu, ok);
       tc_fence_after();
     }
-#pragma unroll
-    for (int which = 0; which < 2; ++which) {
-      const uint32_t col = which ? colDK : colDV;
-      const float mul = which ? p.scale : 1.f;
-      uint8_t* stage = smem + (which ? C::kKOff : C::kVOff);
+    {
+      const uint32_t col = ch ? colDK : colDV;
+      const float mul = ch ? p.scale : 1.f;
+      uint8_t* stage = smem + (ch ? C::kKOff : C::kVOff);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t ov[32];
@@ -344,8 +403,8 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
     fence_proxy_async_smem();
-    named_bar_sync(1, 128);
-    if (r == 0) {
+    named_bar_sync(1, 256);
+    if (threadIdx.x == 0) {
 #pragma unroll
       for (int hf = 0; hf < C::kHalves; ++hf) {
         tma_store_4d(&tm_dv, sb + C::kVOff + hf * C::kAtomBytes, 64 * hf, g, k0, b);
@@ -358,7 +417,7 @@ __global__ void __launch_bounds__(192, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
@@ -369,7 +428,7 @@ __global__ void __launch_bounds__(192, 1)
 // dQ: one CTA per 128-row Q tile; row r = (token t0 + r / Gp, head h0 + r % Gp).
 // ---------------------------------------------------------------------------------------
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
                      const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v,
@@ -382,8 +441,8 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t sb = smem_u32(smem);
   auto bar = [&](int idx) { return sb + C::kQBarOff + 8u * idx; };
   constexpr int kBarIn = 0, kBarKVFull = 1, kBarKVEmpty = 1 + C::kQStages;
-  constexpr int kBarS = 1 + 2 * C::kQStages, kBarP = kBarS + 1, kBarO = kBarS + 2,
-                kBarDrain = kBarS + 3;
+  constexpr int kBarSDP = 1 + 2 * C::kQStages, kBarFree = kBarSDP + 1, kBarDS = kBarSDP + 2,
+                kBarDQ = kBarSDP + 3, kBarO = kBarSDP + 4, kBarDrain = kBarSDP + 5;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kQMiscOff);
   int* abort_flag = reinterpret_cast<int*>(smem + C::kQMiscOff + 4);
   const WaitCtl ctl{abort_flag, p.timeout_ns};
@@ -414,11 +473,12 @@ __global__ void __launch_bounds__(192, 1)
   const int n_kt = jhi - jlo;
 
   if (threadIdx.x == 0) {
-    for (int x = 0; x < C::kQNumBars; ++x) mbar_init(bar(x), (x == kBarP) ? 128 : 1);
+    for (int x = 0; x < C::kQNumBars; ++x)
+      mbar_init(bar(x), (x == kBarFree || x == kBarDS) ? 256 : 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
     tmem_relinquish();
   }
@@ -426,9 +486,9 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  constexpr uint32_t colS = 0, colDP = 128, colDQ = 256;
+  constexpr uint32_t colS = 0, colDP = 128, colDQ = 256, colDS = 384;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ============ producer ============
     if (lane == 0 && n_kt > 0) {
       // (with no key tile the epilogue writes zeros into the Q tile: nothing may land there)
@@ -465,7 +525,7 @@ __global__ void __launch_bounds__(192, 1)
         mbar_wait(bar(kBarKVFull + s), (lastp / C::kQStages) & 1, drain_ctl);
       }
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ============ MMA issuer ============
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
@@ -483,27 +543,40 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
         return r;
       };
+      // Order: S(0) dP(0) | S(t+1) dP(t+1) once S(t), dP(t) are in registers | dQ(t) once
+      // dS(t) is in TMEM: the next tile's products overlap the elementwise work on this one.
+      auto tile_addr = [&](int pos) {
+        return sb + C::kQKVOff + (pos % C::kQStages) * C::kTileBytes;
+      };
+      auto issue_sdp = [&](int t) -> bool {
+        if (!kv_wait(2 * t)) return false;
+        mma_rows(colS, sb + C::kQOff, tile_addr(2 * t));       // S = Q K^T
+        if (!kv_wait(2 * t + 1)) return false;
+        mma_rows(colDP, sb + C::kDOOff, tile_addr(2 * t + 1));  // dP = dO V^T
+        tc_commit(bar(kBarSDP));
+        tc_commit(bar(kBarKVEmpty + (2 * t + 1) % C::kQStages));  // V(t) is done
+        return true;
+      };
       bool ok = n_kt > 0 && mbar_wait(bar(kBarIn), 0, ctl);
       tc_fence_after();
+      if (ok) ok = issue_sdp(0);
       for (int t = 0; t < n_kt && ok; ++t) {
-        const int kpos = 2 * t, vpos = kpos + 1;
-        const uint32_t kt = sb + C::kQKVOff + (kpos % C::kQStages) * C::kTileBytes;
-        const uint32_t vt = sb + C::kQKVOff + (vpos % C::kQStages) * C::kTileBytes;
-        if (!(ok = kv_wait(kpos))) break;
-        mma_rows(colS, sb + C::kQOff, kt);    // S = Q K^T
-        if (!(ok = kv_wait(vpos))) break;
-        mma_rows(colDP, sb + C::kDOOff, vt);  // dP = dO V^T
-        tc_commit(bar(kBarS));
-        tc_commit(bar(kBarKVEmpty + vpos % C::kQStages));
-        if (!(ok = mbar_wait(bar(kBarP), t & 1, ctl))) break;
+        if (t + 1 < n_kt) {
+          if (!(ok = mbar_wait(bar(kBarFree), t & 1, ctl))) break;
+          tc_fence_after();
+          if (!(ok = issue_sdp(t + 1))) break;
+        }
+        if (!(ok = mbar_wait(bar(kBarDS), t & 1, ctl))) break;
         tc_fence_after();
         // dQ += dS K (K tile as the MN-major B operand)
+        const uint32_t kt = tile_addr(2 * t);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tmem + colDQ, tmem + colS + kk * 8,
+          umma_ts(tmem + colDQ, tmem + colDS + kk * 8,
                   smem_desc_sw128(kt + kk * 16 * 128, C::kAtomBytes, 1024), idesc_acc,
                   (t == 0 && kk == 0) ? 0u : 1u);
-        tc_commit(bar(kBarKVEmpty + kpos % C::kQStages));
+        tc_commit(bar(kBarDQ));
+        tc_commit(bar(kBarKVEmpty + (2 * t) % C::kQStages));
       }
       tc_commit(bar(kBarO));
       tc_commit(bar(kBarDrain));
@@ -512,14 +585,16 @@ __global__ void __launch_bounds__(192, 1)
       mbar_wait(bar(kBarDrain), 0, drain_ctl);
     }
   } else {
-    // ============ elementwise: thread = Q row ============
-    const int r = threadIdx.x;
+    // ============ elementwise: thread = Q row; this warp's half of the key columns ============
+    const int wq = warp & 3, ch = warp >> 2;
+    const int r = 32 * wq + lane;
     const int i = tok0 + r / p.Gp;
     const int hh = h0 + r % p.Gp;
-    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * warp) << 16);
-    const float sl2 = p.scale_log2;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * wq) << 16);
+    const uint64_t sl2 = f2(p.scale_log2, p.scale_log2);
     const size_t vrow = (static_cast<size_t>(b) * p.Hq + hh) * p.Sq_pad + min(i, p.Sq_pad - 1);
-    const float l2 = p.lse2[vrow], dlt = p.delta[vrow];
+    const float nl2 = p.lse2[vrow], ndl = p.delta[vrow];  // -L log2(e), -D
+    const uint64_t nl2x2 = f2(nl2, nl2), ndlx2 = f2(ndl, ndl);
     const int ip = i + off;
     const int my_lo = p.window > 0 ? max(0, ip - p.window + 1) : 0;
     const int my_hi = p.causal ? min(ip, p.Skv - 1) : p.Skv - 1;
@@ -528,40 +603,51 @@ __global__ void __launch_bounds__(192, 1)
     const int hi_first = p.causal ? min(first + off, p.Skv - 1) : p.Skv - 1;
     for (int t = 0; t < n_kt; ++t) {
       const int j = jlo + t;
-      bool ok = mbar_wait(bar(kBarS), t & 1, ctl);
+      bool ok = mbar_wait(bar(kBarSDP), t & 1, ctl);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       const bool need_mask = (128 * j < lo_last) || (128 * j + 127 > hi_first) || i >= p.Sq;
+      uint32_t ds[32];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t sv[2][32], dv[2][32];
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          tmem_ld32(trow + colS + 64 * half + 32 * c, sv[c]);
-          tmem_ld32(trow + colDP + 64 * half + 32 * c, dv[c]);
-        }
+      for (int cc = 0; cc < 2; ++cc) {
+        uint32_t sv[32], dv[32];
+        tmem_ld32(trow + colS + 64 * ch + 32 * cc, sv);
+        tmem_ld32(trow + colDP + 64 * ch + 32 * cc, dv);
         tmem_wait_ld();
-        uint32_t ds[32];
 #pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          float dsv[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int col = 2 * x + e;
-            const int key = 128 * j + 64 * half + col;
-            float pr = ex2(fmaf(__uint_as_float(sv[col / 32][col % 32]), sl2, -l2));
-            if (need_mask && (key < my_lo || key > my_hi || i >= p.Sq)) pr = 0.f;
-            dsv[e] = pr * (__uint_as_float(dv[col / 32][col % 32]) - dlt);
+        for (int x = 0; x < 16; ++x) {
+          float a0, a1;
+          f2_split(f2_fma(f2(__uint_as_float(sv[2 * x]), __uint_as_float(sv[2 * x + 1])), sl2,
+                          nl2x2), a0, a1);
+          float p0 = ex2(a0), p1 = ex2(a1);
+          if (need_mask) {
+            const int key = 128 * j + 64 * ch + 32 * cc + 2 * x;
+            if (key < my_lo || key > my_hi || i >= p.Sq) p0 = 0.f;
+            if (key + 1 < my_lo || key + 1 > my_hi || i >= p.Sq) p1 = 0.f;
           }
-          ds[x] = pack_bf16x2(dsv[0], dsv[1]);
+          float d0, d1;
+          f2_split(f2_mul(f2(p0, p1), f2_add(f2(__uint_as_float(dv[2 * x]),
+                                                 __uint_as_float(dv[2 * x + 1])), ndlx2)),
+                   d0, d1);
+          ds[16 * cc + x] = pack_bf16x2(d0, d1);
         }
-        tmem_st32(trow + colS + 32 * half, ds);
       }
+      // S and dP of this tile have been read: the next tile's products may start
+      tc_fence_before();
+      mbar_arrive(bar(kBarFree));
+      // the previous dQ product has read its dS before this one is written over it
+      if (t > 0) {
+        ok = mbar_wait(bar(kBarDQ), (t - 1) & 1, ctl);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
+      }
+      tmem_st32(trow + colDS + 32 * ch, ds);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(bar(kBarP));
+      mbar_arrive(bar(kBarDS));
     }
-    // ---- epilogue: scale * dQ -> bf16 -> swizzled smem (the Q tile) -> TMA ----
+    // ---- epilogue: scale * dQ -> bf16 -> swizzled smem (the Q tile) -> TMA; warps 0-3 take
+    // the first half of the head dims, warps 4-7 the second ----
     bool have = false;
     if (n_kt > 0) {
       bool ok = mbar_wait(bar(kBarO), 0, ctl);
@@ -570,7 +656,8 @@ __global__ void __launch_bounds__(192, 1)
     }
     uint8_t* stage = smem + C::kQOff;
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
+    for (int cc = 0; cc < D / 64; ++cc) {
+      const int c = ch * (D / 64) + cc;
       uint32_t ov[32];
       if (have) {
         tmem_ld32(trow + colDQ + 32 * c, ov);
@@ -592,8 +679,8 @@ __global__ void __launch_bounds__(192, 1)
       }
     }
     fence_proxy_async_smem();
-    named_bar_sync(1, 128);
-    if (r == 0 && tok0 < p.Sq) {
+    named_bar_sync(1, 256);
+    if (threadIdx.x == 0 && tok0 < p.Sq) {
 #pragma unroll
       for (int hf = 0; hf < C::kHalves; ++hf)
         tma_store_4d(&tm_dq, sb + C::kQOff + hf * C::kAtomBytes, 64 * hf, h0, tok0, b);
@@ -604,7 +691,7 @@ __global__ void __launch_bounds__(192, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
