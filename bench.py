@@ -40,8 +40,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from ncu, keyed by the sha256 of the
 # kernel sources they were taken on; a kernel edited since then reports traffic = null.
 NCU_TRAFFIC = {
-    # profiles/fa_prefill_kernel_mha_causal.md: 543.66 MB read + 48.50 MB written, one launch
-    "prefill": {"24eb617e09b98e34": 592_165_120},
+    # profiles/fa_prefill_kernel_mha_causal.md: 534,404,096 B read + 48,113,664 B written
+    "prefill": {"20de4aba3fccfa27": 582_517_760},
     # profiles/fa_decode_split_kernel_decode_int8.md: 1,107,554,560 B read + 8,284,160 B written
     "decode": {"d71c958934a45622": 1_115_838_720},
     # profiles/fa_decode_split_kernel_decode_int8_paged.md: 424,228,864 B read + 6,737,152 B written
@@ -370,6 +370,36 @@ def run_reference(args):
     return 0
 
 
+def run_only_prefill(args):
+    """fa_fwd on the MHA causal workload alone, one JSON line (used to profile the prefill
+    kernel without the other workloads resident on the device)."""
+    import torch
+
+    import synthetic
+    import tiled_attention_26_b200 as fa
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    w = synthetic.WORKLOADS["mha_causal"]
+    q, k, v = synthetic.make_qkv_torch(w, dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=dev)
+    ms = time_calls(torch, stream, lambda: fa.fa_fwd(q, k, v, causal=True, scale=w.scale, o=o,
+                                                      lse=lse, stream=stream),
+                    args.steps, args.warmup)
+    if fa.fa_device_status() != 0:
+        raise RuntimeError("the prefill kernel reported a device-side error")
+    flops = prefill_flops(w)
+    peaks, _ = load_peaks()
+    print(json.dumps({"metric": "attention forward TFLOP/s (4*D flops per visible pair)",
+                      "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                      "ms_per_call": ms, "steps": args.steps, "warmup": args.warmup,
+                      "frac_of_burst": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                      "config": {"workload": "mha_causal (B=2, H=32, S=4096, D=128, causal)"}}),
+          flush=True)
+    return 0
+
+
 def run_only_backward(args):
     """fa_bwd on the MHA causal workload alone, one JSON line (used to profile the backward
     kernels without the other workloads resident on the device)."""
@@ -401,13 +431,15 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["backward"], default=None,
+    ap.add_argument("--only", choices=["backward", "prefill"], default=None,
                     help="time one further row on its own (for profiling); prints its own line")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
     if args.only == "backward":
         return run_only_backward(args)
+    if args.only == "prefill":
+        return run_only_prefill(args)
 
     import torch
 
