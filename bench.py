@@ -370,6 +370,62 @@ def run_reference(args):
     return 0
 
 
+class Ranks:
+    """One process per GPU: rank / world from the torchrun environment, a process group when
+    world > 1 (nccl on GPUs; the tests use gloo), a barrier, and the max over ranks that every
+    reported time goes through.  Every rank runs its own independent workload, so no data-path
+    collective exists: the only collectives are the barrier and these max-reductions."""
+
+    def __init__(self, world: int, rank: int, local: int, backend: str | None):
+        import torch
+        self.world, self.rank, self.local = world, rank, local
+        self.dist = None
+        self.device = "cpu"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            self.device = torch.device("cuda", local)
+        if world > 1:
+            import datetime
+
+            import torch.distributed as dist
+            kw = {"device_id": self.device} if backend == "nccl" else {}
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120), **kw)
+            self.dist = dist
+
+    @classmethod
+    def from_env(cls, backend: str):
+        return cls(int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")),
+                   int(os.environ.get("LOCAL_RANK", "0")), backend)
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+    def max(self, x: float) -> float:
+        if self.dist is None:
+            return float(x)
+        import torch
+        t = torch.tensor([float(x)], dtype=torch.float64, device=self.device)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.dist is not None:
+            self.dist.destroy_process_group()
+            self.dist = None
+
+
+def rank_seed_offset(rank: int) -> int:
+    """Rank r draws its inputs from seeds shifted by 1000 r: independent problems per GPU."""
+    return 1000 * rank
+
+
+def weak_scaling_throughput(world: int, steps: int, work_per_step: float, max_ms: float) -> float:
+    """Whole-job throughput (work units per second): every rank did `steps` steps of
+    `work_per_step` units; the job took the slowest rank's time."""
+    return world * steps * work_per_step / (max_ms * 1e-3)
+
+
 def run_only_prefill(args):
     """fa_fwd on the MHA causal workload alone, one JSON line (used to profile the prefill
     kernel without the other workloads resident on the device)."""
@@ -446,33 +502,14 @@ def main():
     import synthetic
     import tiled_attention_26_b200 as fa
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    torch.cuda.set_device(local)
-    dist = None
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
-
-    def max_over_ranks(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    ranks = Ranks.from_env("nccl")
+    world, rank, local = ranks.world, ranks.rank, ranks.local
+    barrier, max_over_ranks = ranks.barrier, ranks.max
 
     wp = synthetic.WORKLOADS["mha_causal"]
     wd = synthetic.WORKLOADS["decode_int8"]
     dev = torch.device("cuda", local)
-    seed_off = 1000 * rank
+    seed_off = rank_seed_offset(rank)
     q = synthetic.normal_bf16_torch(wp.seed(0) + seed_off, wp.q_shape(), dev)
     k = synthetic.normal_bf16_torch(wp.seed(1) + seed_off, wp.kv_shape(), dev)
     v = synthetic.normal_bf16_torch(wp.seed(2) + seed_off, wp.kv_shape(), dev)
@@ -537,8 +574,8 @@ def main():
     flops = prefill_flops(wp)
     dbytes = decode_bytes(wd)
     peaks, peak_src = load_peaks()
-    pre_tflops = world * K * flops / (pre_sum * 1e-3) / 1e12
-    dec_gbs = world * K * dbytes / (dec_sum * 1e-3) / 1e9
+    pre_tflops = weak_scaling_throughput(world, K, flops, pre_sum) / 1e12
+    dec_gbs = weak_scaling_throughput(world, K, dbytes, dec_sum) / 1e9
     pre_avg_s = sum(pre_ms) / K * 1e-3
     dec_avg_s = sum(dec_ms) / K * 1e-3
     achieved = flops / pre_avg_s / 1e12
@@ -589,9 +626,10 @@ def main():
         barrier()
         p_ms = max_over_ranks(sum(e3[s][0].elapsed_time(e3[s][1]) for s in range(E)))
         d_ms = max_over_ranks(sum(e3[s][1].elapsed_time(e3[s][2]) for s in range(E)))
-        e2e = {"value": world * E * flops / (p_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": weak_scaling_throughput(world, E, flops, p_ms) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": E,
-               "decode": {"value": world * E * dbytes / (d_ms * 1e-3) / 1e9, "unit": "GB/s"},
+               "decode": {"value": weak_scaling_throughput(world, E, dbytes, d_ms) / 1e9,
+                          "unit": "GB/s"},
                "ms_per_step": (p_ms + d_ms) / E}
 
     cpu = None
@@ -687,8 +725,7 @@ def main():
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
-    if dist is not None:
-        dist.destroy_process_group()
+    ranks.close()
     return 0
 
 
