@@ -683,7 +683,7 @@ def main():
             "paged_decode": {
                 "workload": "decode_int8_paged: B=16, Hq=32, Hkv=8, D=128, INT8 KV in 64-token "
                             "pages scattered over the pool, lengths uniform in [1, 32768] "
-                            f"({pg_bytes / 1e6:.1f} MB per call), 16 splits",
+                            f"({pg_bytes / 1e6:.1f} MB per call), 8 splits",
                 "kernel": "fa_decode_split_kernel<128, paged> + fa_decode_combine_kernel<128>",
                 "ms_per_call": pg_ms, "achieved": pg_bytes / (pg_ms * 1e-3) / 1e9,
                 "unit": "GB/s", "peak": peaks["hbm_gbs"],

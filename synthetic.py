@@ -343,7 +343,7 @@ class PagedDecodeWorkload:
 
 PAGED_WORKLOADS = {
     "decode_int8_paged": PagedDecodeWorkload(
-        "decode_int8_paged", 6, 16, 32, 8, 128, 64, 1, 32768, 16,
+        "decode_int8_paged", 6, 16, 32, 8, 128, 64, 1, 32768, 8,
         note="GQA decode over a paged INT8 cache, lengths uniform in [1, 32768]"),
 }
 

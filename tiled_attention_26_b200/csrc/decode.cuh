@@ -159,6 +159,10 @@ __device__ __forceinline__ void cp_async_wait_all() {
 #define FA_DECODE_STAGES 2  // K/V stages of 128 keys in the shared-memory ring (3 CTAs per SM)
 #endif
 
+#ifndef FA_DECODE_MIN_CHUNK
+#define FA_DECODE_MIN_CHUNK 128  // keys; a multiple of 128
+#endif
+
 #ifndef FA_DECODE_PDL
 #define FA_DECODE_PDL 1  // launch the merge kernel as a programmatic dependent of the split kernel
 #endif
@@ -250,8 +254,10 @@ __global__ void __launch_bounds__(160, 1) fa_decode_split_kernel(
       len = max(0, min(len, cap));
     }
   }
-  // splits are whole stages: every stage starts on a multiple of 128 keys
-  const int chunk = ((len + p.splits - 1) / p.splits + C::kT - 1) / C::kT * C::kT;
+  // splits are whole stages (every stage starts on a multiple of 128 keys) of at least
+  // FA_DECODE_MIN_CHUNK keys: a short sequence takes few splits rather than many tiny ones
+  const int chunk = max(FA_DECODE_MIN_CHUNK,
+                        ((len + p.splits - 1) / p.splits + C::kT - 1) / C::kT * C::kT);
   const int t_begin = min(len, split * chunk);
   const int t_end = min(len, t_begin + chunk);
   const int n_stages = (t_end - t_begin + C::kT - 1) / C::kT;
