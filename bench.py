@@ -42,9 +42,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC = {
     # profiles/fa_prefill_kernel_mha_causal.md: 534,404,096 B read + 48,113,664 B written
     "prefill": {"20de4aba3fccfa27": 582_517_760},
-    # profiles/fa_decode_split_kernel_decode_int8.md: 1,107,554,560 B read + 8,284,160 B written
-    "decode": {"d71c958934a45622": 1_115_838_720},
-    # profiles/fa_decode_split_kernel_decode_int8_paged.md: 424,228,864 B read + 6,737,152 B written
+    # profiles/fa_decode_split_kernel_decode_int8.md: 1,107,567,616 B read + 6,939,648 B written
+    "decode": {"0374b3d7a3500c43": 1_114_507_264},
+    # profiles/fa_decode_split_kernel_decode_int8_paged.md (earlier source of the same kernel)
     "paged_decode": {"d71c958934a45622": 430_966_016},
 }
 

@@ -201,12 +201,20 @@ __device__ __forceinline__ uint32_t swz(uint32_t off) {
   else return off;
 }
 
-// INT4: nibbles at bits [s, s+4) and [s+16, s+20) of an offset-binary word (code + 8) -> fp16x2
-// {code_lo, code_hi} exactly: 1024 + n in fp16 has unit mantissa steps, minus 1032 leaves n - 8.
-__device__ __forceinline__ uint32_t nibbles_to_f16x2(uint32_t biased, int s) {
-  const uint32_t h = ((biased >> s) & 0x000F000Fu) | 0x64006400u;
+// INT4 codes of an offset-binary word (code + 8 per nibble) -> fp16x2, exactly.  In fp16 with
+// exponent 2^10 the mantissa counts units, so: nibbles at bits [0,4) and [16,20) give 1024 + n,
+// minus 1032 leaves n - 8; nibbles at bits [4,8) and [20,24) give 1024 + 16 n, minus 1152
+// leaves 16 (n - 8), scaled by 16 (the caller folds 1/16 into the other operand or the output).
+__device__ __forceinline__ uint32_t nib_lo_f16x2(uint32_t biased) {
+  const uint32_t h = (biased & 0x000F000Fu) | 0x64006400u;
   uint32_t d;
   asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(h), "r"(0x64086408u));
+  return d;
+}
+__device__ __forceinline__ uint32_t nib_hi16_f16x2(uint32_t biased) {
+  const uint32_t h = (biased & 0x00F000F0u) | 0x64006400u;
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(h), "r"(0x64806480u));
   return d;
 }
 
@@ -388,10 +396,13 @@ __global__ void __launch_bounds__(160, 1) fa_decode_split_kernel(
     amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
     const int eq = pow2_exponent_below(amax, 15);
     const float qs = exp2i(eq);
+    // INT4: the K fragment's second pair of each k-step carries 16 x the code (nib_hi16), so
+    // its Q partner is scaled by 1/16 (exact)
+    const float qs_hi = kBits == 4 ? qs * 0.0625f : qs;
 #pragma unroll
     for (int s = 0; s < KS; ++s) {
       qf[s][0] = pack_f16x2(qv[s][0] * qs, qv[s][1] * qs);
-      qf[s][1] = pack_f16x2(qv[s][2] * qs, qv[s][3] * qs);
+      qf[s][1] = pack_f16x2(qv[s][2] * qs_hi, qv[s][3] * qs_hi);
     }
     sc_mine = p.scale_log2 * exp2i(-eq);
   }
@@ -449,11 +460,11 @@ __global__ void __launch_bounds__(160, 1) fa_decode_split_kernel(
                           codes_to_f16x2(w0, kSelB23), codes_to_f16x2(w1, kSelB23), qf[st][0],
                           qf[st][1]);
           } else {
-            const uint32_t w0 = kw[0][st >> 1], w1 = kw[1][st >> 1];
-            const int sh = 8 * (st & 1);
-            mma_f16_16816(sacc, nibbles_to_f16x2(w0, sh), nibbles_to_f16x2(w1, sh),
-                          nibbles_to_f16x2(w0, sh + 4), nibbles_to_f16x2(w1, sh + 4), qf[st][0],
-                          qf[st][1]);
+            // k-step 2j + h of word j: nibbles (2h, 2h+4) as is, (2h+1, 2h+5) times 16
+            const uint32_t w0 = kw[0][st >> 1] >> (8 * (st & 1));
+            const uint32_t w1 = kw[1][st >> 1] >> (8 * (st & 1));
+            mma_f16_16816(sacc, nib_lo_f16x2(w0), nib_lo_f16x2(w1), nib_hi16_f16x2(w0),
+                          nib_hi16_f16x2(w1), qf[st][0], qf[st][1]);
           }
         }
         const int rA = r_w + 16 * u + g, rB = rA + 8;
@@ -576,13 +587,14 @@ __global__ void __launch_bounds__(160, 1) fa_decode_split_kernel(
           } else {
             const int w = mt >> 2;
             const uint32_t sel = (mt & 2) ? 0x7632u : 0x5410u;
-            const uint32_t x01 = prmt(r[0][w], r[1][w], sel);  // [k0.b, k0.b', k1.b, k1.b']
-            const uint32_t x89 = prmt(r[2][w], r[3][w], sel);
-            const int sh = 8 * (mt & 1);
-            a0 = nibbles_to_f16x2(x01, sh);
-            a1 = nibbles_to_f16x2(x01, sh + 4);
-            a2 = nibbles_to_f16x2(x89, sh);
-            a3 = nibbles_to_f16x2(x89, sh + 4);
+            // [k0.b, k0.b', k1.b, k1.b'], shifted so that this m-tile's byte is the low one
+            const uint32_t x01 = prmt(r[0][w], r[1][w], sel) >> (8 * (mt & 1));
+            const uint32_t x89 = prmt(r[2][w], r[3][w], sel) >> (8 * (mt & 1));
+            // dim 2mt (low nibble) as is; dim 2mt+1 (high nibble) times 16, undone at the end
+            a0 = nib_lo_f16x2(x01);
+            a1 = nib_hi16_f16x2(x01);
+            a2 = nib_lo_f16x2(x89);
+            a3 = nib_hi16_f16x2(x89);
           }
           mma_f16_16816(oacc[mt], a0, a1, a2, a3, pb[u][0], pb[u][1]);
         }
@@ -609,14 +621,16 @@ __global__ void __launch_bounds__(160, 1) fa_decode_split_kernel(
     sm_l[warp * 8 + 2 * c + 1] = l1;
   }
   const float unscale = (E == kEUnset) ? 0.f : exp2i_or_zero(-E);
+  // INT4: the odd dims (rows g + 8 of each m-tile) were accumulated from 16 x the codes
+  const float unscale_hi = kBits == 4 ? unscale * 0.0625f : unscale;
 #pragma unroll
   for (int mt = 0; mt < MT; ++mt) {
     const int d0 = DPT * g + 2 * mt;
     float* ow = sm_o + warp * 8 * D;
     ow[(2 * c) * D + d0] = oacc[mt][0] * unscale;
     ow[(2 * c + 1) * D + d0] = oacc[mt][1] * unscale;
-    ow[(2 * c) * D + d0 + 1] = oacc[mt][2] * unscale;
-    ow[(2 * c + 1) * D + d0 + 1] = oacc[mt][3] * unscale;
+    ow[(2 * c) * D + d0 + 1] = oacc[mt][2] * unscale_hi;
+    ow[(2 * c + 1) * D + d0 + 1] = oacc[mt][3] * unscale_hi;
   }
   named_bar_sync(1, 128);
   for (int idx = threadIdx.x; idx < nheads * D; idx += 128) {
