@@ -145,7 +145,8 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
 
   auto kernel = fa::fa_prefill_kernel<D, kMode>;
   const int variant = (D == 128 ? 4 : 0) + kMode;
-  if ((rc = ensure_smem_attr(kernel, C::kSmemBytes, g_attr_prefill[variant])) != FA_OK) return rc;
+  constexpr int smem_bytes = (kMode & fa::kModeMask) ? C::kSmemBytesMask : C::kSmemBytes;
+  if ((rc = ensure_smem_attr(kernel, smem_bytes, g_attr_prefill[variant])) != FA_OK) return rc;
   // The kernel redistributes its launch registers between warpgroups (setmaxnreg); that only
   // completes if the launch gave every thread at least kMinLaunchRegs.
   int regs = g_prefill_regs[variant].load(std::memory_order_acquire);
@@ -156,7 +157,7 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
     g_prefill_regs[variant].store(regs, std::memory_order_release);
   }
   if (regs < C::kMinLaunchRegs) return FA_ERR_UNSUPPORTED;
-  kernel<<<static_cast<unsigned>(grid), C::kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, to, p);
+  kernel<<<static_cast<unsigned>(grid), C::kThreads, smem_bytes, stream>>>(tq, tk, tv, to, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

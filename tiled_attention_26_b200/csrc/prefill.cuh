@@ -99,6 +99,13 @@ struct PrefillCfg {
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + slack to align the base
+  // mask variant: per softmax warp, two 16-key chunks of its 32 rows' mask (fp32), staged
+  // by asynchronous copies
+  static constexpr int kMaskChunk = 16;
+  static constexpr int kMaskSlotBytes = 32 * kMaskChunk * 4;  // 2 KB
+  static constexpr int kMaskOff = (kMiscOff + 16 + 127) / 128 * 128;
+  static constexpr int kMaskBytes = 8 * 2 * kMaskSlotBytes;   // 32 KB
+  static constexpr int kSmemBytesMask = kMaskOff + kMaskBytes + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kRegsSoftmax = FA_REGS_SOFTMAX;
   // the rest of the 384 x 168 launch registers go to the producer / MMA warpgroup
@@ -459,12 +466,59 @@ __global__ void __launch_bounds__(384, 1)
     const int my_lo = vis_lo(p, i), my_hi = vis_hi(p, i);
     const int t_last_tok = min(tok0 + t * tpt + tpt, p.Sq) - 1;
     const float sl2 = p.scale_log2;
-    // this row's mask, or null (no mask, or a padding row past Sq)
-    const float* mrow = nullptr;
+    const bool mvec = p.mask_vec != 0;  // rows start 16-byte aligned: staged vector copies
+    // Mask staging (kMask, mvec): this warp's 32 rows, 16 keys at a time, copied with 16-byte
+    // cp.async (lane: row (lane >> 2) + 8 it, bytes 16 (lane & 3)) into two 2 KB slots; a row's
+    // 16-byte pieces sit at (row, piece ^ ((row >> 1) & 3)) so that the row-per-lane reads
+    // spread over all banks.  Chunk number mseq runs across tiles; chunk 0 of the next tile is
+    // requested while this tile's last chunk is read.
+    int mseq = 0;
+    // the first of the four rows this lane copies (the others follow 8 rows apart)
+    const int crow0 = t * 128 + 32 * (warp & 3) + (lane >> 2);
+    uint8_t* const mbase = smem + C::kMaskOff + warp * 2 * C::kMaskSlotBytes;
+    auto mslot = [&](int slot) -> const uint8_t* { return mbase + slot * C::kMaskSlotBytes; };
+    // copy chunk k (keys 16k.. of key tile jt) into slot `slot`
+    auto mask_issue = [&](int jt, int k, int slot) {
+#pragma unroll
+      for (int it = 0; it < 4; ++it) {
+        const int row = (lane >> 2) + 8 * it, pc = lane & 3;
+        const int key = 128 * jt + C::kMaskChunk * k + 4 * pc;
+        const int Rr = crow0 + 8 * it;
+        const int ir = tok0 + Rr / p.Gp, hr = h0 + Rr % p.Gp;
+        const bool ok = ir < p.Sq && key < p.Skv;
+        const float* src = ok ? p.mask + b * p.mask_sb + hr * p.mask_sh +
+                                    static_cast<long long>(ir) * p.Skv + key
+                              : p.mask;
+        const uint32_t dst = smem_u32(mbase + slot * C::kMaskSlotBytes + row * 64 +
+                                      16 * (pc ^ ((row >> 1) & 3)));
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                     "r"(ok ? 16 : 0)
+                     : "memory");
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    // next needed key tile of this Q tile after jt (or -1)
+    auto next_tile = [&](int jt) -> int {
+      for (int x = jt + 1; x <= my_ts.last; ++x)
+        if (my_ts.has<kGlobal>(x, gT)) return x;
+      return -1;
+    };
+    // before reading chunk k of tile jt (chunk number mseq): request the following chunk, then
+    // wait until this one has landed
+    auto mask_stage = [&](int jt, int k) {
+      bool more = true;
+      if (k + 1 < 128 / C::kMaskChunk) {
+        mask_issue(jt, k + 1, (mseq + 1) & 1);
+      } else {
+        const int jn = next_tile(jt);
+        if (jn >= 0) mask_issue(jn, 0, (mseq + 1) & 1); else more = false;
+      }
+      if (more) asm volatile("cp.async.wait_group 1;" ::: "memory");
+      else asm volatile("cp.async.wait_group 0;" ::: "memory");
+      __syncwarp();
+    };
     if constexpr (kMask)
-      if (i < p.Sq)
-        mrow = p.mask + b * p.mask_sb + hh * p.mask_sh + static_cast<long long>(i) * p.Skv;
-    const bool mvec = p.mask_vec != 0;  // rows start 16-byte aligned: vector loads
+      if (mvec && my_ts.last >= my_ts.first) mask_issue(my_ts.first, 0, 0);
     float m = -INFINITY, l = 0.f;
     int n = 0;
     for (int j = my_ts.first; j <= my_ts.last; ++j) {
@@ -479,23 +533,39 @@ __global__ void __launch_bounds__(384, 1)
       tmem_wait_ld();
       if constexpr (kMask) {
         // scores += mask / scale (the exponent then carries scale * s + mask, in log2 units)
-        if (mrow != nullptr) {
+        if (mvec) {
+          // the mask chunks were staged in shared memory by coalesced asynchronous copies
+#pragma unroll
+          for (int k = 0; k < 128 / C::kMaskChunk; ++k) {
+            mask_stage(j, k);  // issues the next chunk, waits for this one
+#pragma unroll
+            for (int pc = 0; pc < 4; ++pc) {
+              const float4 x = *reinterpret_cast<const float4*>(
+                  mslot(mseq & 1) + (r & 31) * 64 + 16 * (pc ^ (((r & 31) >> 1) & 3)));
+              const float mv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int col = C::kMaskChunk * k + 4 * pc + e;
+                sv[col / 32][col % 32] = __float_as_uint(
+                    fmaf(mv[e], p.inv_scale, __uint_as_float(sv[col / 32][col % 32])));
+              }
+            }
+            __syncwarp();  // every lane has read the slot before it is refilled
+            ++mseq;
+          }
+        } else if (i < p.Sq) {
+          // rows not 16-byte aligned: this row's values, one at a time
+          const float* mrow =
+              p.mask + b * p.mask_sb + hh * p.mask_sh + static_cast<long long>(i) * p.Skv;
 #pragma unroll
           for (int c = 0; c < 4; ++c)
 #pragma unroll
             for (int q4 = 0; q4 < 8; ++q4) {
               const int key = 128 * j + 32 * c + 4 * q4;
               float mv[4] = {0.f, 0.f, 0.f, 0.f};
-              if (mvec) {
-                if (key < p.Skv) {
-                  const float4 x = __ldg(reinterpret_cast<const float4*>(mrow + key));
-                  mv[0] = x.x; mv[1] = x.y; mv[2] = x.z; mv[3] = x.w;
-                }
-              } else {
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  if (key + e < p.Skv) mv[e] = __ldg(mrow + key + e);
-              }
+              for (int e = 0; e < 4; ++e)
+                if (key + e < p.Skv) mv[e] = __ldg(mrow + key + e);
 #pragma unroll
               for (int e = 0; e < 4; ++e)
                 sv[c][4 * q4 + e] = __float_as_uint(
@@ -569,6 +639,9 @@ __global__ void __launch_bounds__(384, 1)
       l = l * alpha + ((a0 + a1) + (a2 + a3));
       ++n;
     }
+
+    // mask copies still in flight (after an abandoned wait) land before the CTA moves on
+    if constexpr (kMask) asm volatile("cp.async.wait_all;" ::: "memory");
 
     // ---- epilogue: O / l -> bf16 -> shared memory (swizzled like the O tensor map) -> TMA ----
     bool have_o = false;
