@@ -70,9 +70,9 @@ struct BwdCfg {
   static constexpr int kVOff = kTileBytes;
   static constexpr int kUOff = 2 * kTileBytes;
   static constexpr int kUBarOff = kUOff + kUStages * kUnitBytes;
-  // barriers: kv_full, u_full[S], u_empty[S], s_full, dp_full, p_ready, ds_ready, o_final,
-  // drain
-  static constexpr int kUNumBars = 7 + 2 * kUStages;
+  // barriers: kv_full, u_full[S] (Q and the vectors), u_empty[S], s_full, dp_full, p_ready,
+  // ds_ready, o_final, drain, u_do[S] (dO)
+  static constexpr int kUNumBars = 7 + 3 * kUStages;
   static constexpr int kUMiscOff = kUBarOff + 8 * kUNumBars;
   static constexpr int kUSmemBytes = kUMiscOff + 16 + 1024;
 };
@@ -144,7 +144,8 @@ __global__ void __launch_bounds__(320, 1)
   auto bar = [&](int idx) { return sb + C::kUBarOff + 8u * idx; };
   constexpr int kBarKV = 0, kBarUFull = 1, kBarUEmpty = 1 + C::kUStages;
   constexpr int kBarS = 1 + 2 * C::kUStages, kBarDP = kBarS + 1, kBarP = kBarS + 2,
-                kBarDS = kBarS + 3, kBarO = kBarS + 4, kBarDrain = kBarS + 5;
+                kBarDS = kBarS + 3, kBarO = kBarS + 4, kBarDrain = kBarS + 5,
+                kBarUDo = kBarS + 6;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kUMiscOff);
   int* abort_flag = reinterpret_cast<int*>(smem + C::kUMiscOff + 4);
   const WaitCtl ctl{abort_flag, p.timeout_ns};
@@ -205,18 +206,21 @@ __global__ void __launch_bounds__(320, 1)
           break;
         const int h = g * p.G + u / n_qt, i0 = 128 * (qt_lo + u % n_qt);
         const uint32_t base = sb + C::kUOff + s * C::kUnitBytes;
-        mbar_arrive_expect_tx(bar(kBarUFull + s), C::kUnitBytes);
+        // Q and the vectors first (S^T needs them), dO on a barrier of its own (dP^T)
+        mbar_arrive_expect_tx(bar(kBarUFull + s), C::kTileBytes + 1024);
 #pragma unroll
-        for (int hf = 0; hf < C::kHalves; ++hf) {
+        for (int hf = 0; hf < C::kHalves; ++hf)
           tma_load_4d(base + hf * C::kAtomBytes, &tm_q, bar(kBarUFull + s), 64 * hf, h, i0, b);
-          tma_load_4d(base + C::kTileBytes + hf * C::kAtomBytes, &tm_do, bar(kBarUFull + s),
-                      64 * hf, h, i0, b);
-        }
         // L and D vectors: rows (b*Hq + h) of the two [B*Hq, Sq_pad] workspace arrays, which
         // the vector map sees as one (Sq_pad, B*Hq, 2) tensor
         const uint32_t vb = base + 2 * C::kTileBytes;
         tma_load_3d(vb, &tm_vec, bar(kBarUFull + s), i0, b * p.Hq + h, 0);
         tma_load_3d(vb + 512, &tm_vec, bar(kBarUFull + s), i0, b * p.Hq + h, 1);
+        mbar_arrive_expect_tx(bar(kBarUDo + s), C::kTileBytes);
+#pragma unroll
+        for (int hf = 0; hf < C::kHalves; ++hf)
+          tma_load_4d(base + C::kTileBytes + hf * C::kAtomBytes, &tm_do, bar(kBarUDo + s),
+                      64 * hf, h, i0, b);
         issued = u + 1;
       }
       volatile int zero = 0;
@@ -225,6 +229,7 @@ __global__ void __launch_bounds__(320, 1)
       for (int s = 0; s < C::kUStages && s < issued; ++s) {
         const int last = s + C::kUStages * ((issued - 1 - s) / C::kUStages);
         mbar_wait(bar(kBarUFull + s), (last / C::kUStages) & 1, drain_ctl);
+        mbar_wait(bar(kBarUDo + s), (last / C::kUStages) & 1, drain_ctl);
       }
     }
   } else if (warp == 9) {
@@ -265,8 +270,11 @@ __global__ void __launch_bounds__(320, 1)
         unit_tiles(0, qt, dot);
         mma_rows(colS, sb + C::kKOff, qt);    // S^T = K Q^T
         tc_commit(bar(kBarS));
-        mma_rows(colDP, sb + C::kVOff, dot);  // dP^T = V dO^T
-        tc_commit(bar(kBarDP));
+        if ((ok = mbar_wait(bar(kBarUDo), 0, ctl))) {
+          tc_fence_after();
+          mma_rows(colDP, sb + C::kVOff, dot);  // dP^T = V dO^T
+          tc_commit(bar(kBarDP));
+        }
       }
       for (int u = 0; u < n_units && ok; ++u) {
         uint32_t qt, dot, qn = 0, don = 0;
@@ -288,6 +296,9 @@ __global__ void __launch_bounds__(320, 1)
         mma_acc(colDK, colDP, qt, u == 0);    // dK += dS^T Q
         tc_commit(bar(kBarUEmpty + u % C::kUStages));
         if (nxt) {
+          if (!(ok = mbar_wait(bar(kBarUDo + (u + 1) % C::kUStages), ((u + 1) / C::kUStages) & 1, ctl)))
+            break;
+          tc_fence_after();
           mma_rows(colDP, sb + C::kVOff, don);  // dP^T of the next unit (after dK read dS)
           tc_commit(bar(kBarDP));
         }
