@@ -137,3 +137,19 @@ def test_global_local_brute_force_and_reductions():
     o4, l4 = oracle.attn(q, k, v, 0.125, 1, W)
     np.testing.assert_allclose(o3, o4, atol=1e-15, rtol=0)
     np.testing.assert_allclose(l3, l4, atol=1e-15, rtol=0)
+
+
+@pytest.mark.parametrize("W", [1, 8, 50])
+def test_printed_mask_code_is_window_w_plus_one(W):
+    # the page builds tril(ones, 0) * triu(ones, -W): it keeps i - W <= j <= i, i.e. W + 1 keys,
+    # which this project's rule reaches as window = W + 1 (its own reading keeps W keys)
+    S = 64
+    q, k, v = _qkv(1, 2, 1, S, S, 64, 81 + W)
+    ones = np.ones((S, S))
+    keep = np.tril(ones, 0) * np.triu(ones, -W)
+    mask = np.where(keep > 0, 0.0, -np.inf).astype(np.float32)[None, None]
+    o_page, l_page = oracle.attn_ext(q, k, v, 0.125, 0, 0, 0, mask)
+    o_w1, l_w1 = oracle.attn(q, k, v, 0.125, 1, W + 1)
+    np.testing.assert_allclose(o_page, o_w1, atol=1e-13, rtol=0)
+    np.testing.assert_allclose(l_page, l_w1, atol=1e-13, rtol=0)
+    assert int(keep.sum()) == sum(min(i + 1, W + 1) for i in range(S))

@@ -214,3 +214,29 @@ def test_binding_raises_on_bad_arguments(fa):
     with pytest.raises(fa.FaError) as e:
         fa.fa_fwd(q, q, q, causal=False, window=4)
     assert e.value.status == fa.STATUS["FA_ERR_INVALID_ARG"]
+
+
+def test_decode_equals_prefill_on_representable_kv(fa):
+    # With power-of-two scales, code * scale is exact in bf16, so the INT8 decode of one query
+    # must match the bf16 prefill kernel on the dequantised cache (Sq = 1, bottom-right causal).
+    import torch
+    B, Hq, Hkv, Skv, D = 2, 8, 2, 700, 128
+    rng = np.random.default_rng(12)
+    q = synthetic.normal_bf16(90, (B, 1, Hq, D))
+    codes_k = rng.integers(-127, 128, size=(B, Skv, Hkv, D)).astype(np.int8)
+    codes_v = rng.integers(-127, 128, size=(B, Skv, Hkv, D)).astype(np.int8)
+    ks = (2.0 ** rng.integers(-9, -5, size=(B, Hkv, Skv))).astype(np.float32)
+    vs = (2.0 ** rng.integers(-9, -5, size=(B, Hkv, Skv))).astype(np.float32)
+    kf = codes_k.astype(np.float32) * np.transpose(ks, (0, 2, 1))[..., None]
+    vf = codes_v.astype(np.float32) * np.transpose(vs, (0, 2, 1))[..., None]
+    kb, vb = synthetic.f32_to_bf16_bits(kf), synthetic.f32_to_bf16_bits(vf)
+    assert np.array_equal(synthetic.bf16_bits_to_f32(kb), kf)  # exact
+    s = float(np.float32(1 / math.sqrt(D)))
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).cuda()
+    od, ld = fa.fa_decode_int8(to_dev_bf16(q), dev(codes_k), dev(codes_v), dev(ks), dev(vs),
+                               num_splits=4, scale=s)
+    op, lp = fa.fa_fwd(to_dev_bf16(q), to_dev_bf16(kb), to_dev_bf16(vb), causal=True, scale=s)
+    torch.cuda.synchronize()
+    assert fa.fa_device_status() == 0
+    assert (od.float() - op.float()).abs().max().item() <= 2e-2
+    assert (ld - lp[:, :, 0]).abs().max().item() <= 1e-3
