@@ -40,12 +40,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from ncu, keyed by the sha256 of the
 # kernel sources they were taken on; a kernel edited since then reports traffic = null.
 NCU_TRAFFIC = {
-    # profiles/fa_prefill_kernel_mha_causal.md: 534,404,096 B read + 48,113,664 B written
-    "prefill": {"20de4aba3fccfa27": 582_517_760},
+    # profiles/fa_prefill_kernel_mha_causal.md: 532,551,168 B read + 47,900,160 B written
+    "prefill": {"cf0efa0ff3706f95": 580_451_328},
     # profiles/fa_decode_split_kernel_decode_int8.md: 1,107,567,616 B read + 6,939,648 B written
     "decode": {"0374b3d7a3500c43": 1_114_507_264},
-    # profiles/fa_decode_split_kernel_decode_int8_paged.md (earlier source of the same kernel)
-    "paged_decode": {"d71c958934a45622": 430_966_016},
+    # profiles/fa_decode_split_kernel_decode_int8_paged.md: 424,233,984 B read + 4,904,448 B
+    # written
+    "paged_decode": {"0374b3d7a3500c43": 429_138_432},
 }
 
 
@@ -478,6 +479,28 @@ def run_only_backward(args):
     return 0
 
 
+def run_only_paged(args):
+    """fa_decode_int8_paged on the paged workload alone, one JSON line (used to profile the
+    paged decode kernels without the other workloads resident on the device)."""
+    import torch
+
+    import synthetic
+    import tiled_attention_26_b200 as fa
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    ms, nbytes = measure_paged_decode(fa, synthetic, torch, dev, stream, steps=args.steps,
+                                      warmup=args.warmup)
+    peaks, _ = load_peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    print(json.dumps({"metric": "paged INT8 decode GB/s (algorithmic bytes)", "value": gbs,
+                      "unit": "GB/s", "ms_per_call": ms, "bytes_per_call": nbytes,
+                      "steps": args.steps, "warmup": args.warmup,
+                      "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                      "config": {"workload": "decode_int8_paged"}}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -487,7 +510,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["backward", "prefill"], default=None,
+    ap.add_argument("--only", choices=["backward", "prefill", "paged"], default=None,
                     help="time one further row on its own (for profiling); prints its own line")
     args = ap.parse_args()
     if args.impl == "reference":
@@ -496,6 +519,8 @@ def main():
         return run_only_backward(args)
     if args.only == "prefill":
         return run_only_prefill(args)
+    if args.only == "paged":
+        return run_only_paged(args)
 
     import torch
 

@@ -16,7 +16,9 @@
 //              writes P (bf16) back into TMEM over S, rescales O in TMEM when m grew by more
 //              than 2^8, and at the end normalises O, stages it in shared memory and stores it
 //              with TMA, plus the row's log-sum-exp.
-//   warp 8     TMA producer: Q tiles once, then K_j, V_j into a ring of shared-memory stages.
+//   warp 8     TMA producer: Q tiles once, then K_j, V_j into a ring of shared-memory stages;
+//              both copies of tile j complete on the full barrier of K_j's stage, so the MMA
+//              thread waits once per key tile.
 //   warp 9     allocates TMEM and issues tcgen05.mma from one thread:
 //                S_t = Q_t K_j^T (both operands in shared memory),
 //                O_t += P_t V_j  (P from TMEM, V from shared memory; P arrives in two halves).
@@ -334,20 +336,23 @@ __global__ void __launch_bounds__(384, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(bar(C::kBarKVFull + s), C::kTileBytes);
+          // K_j and V_j land on the full barrier of K_j's stage (an even stage)
+          const int sf = (2 * kt) % C::kStages;
+          if (kind == 0) mbar_arrive_expect_tx(bar(C::kBarKVFull + sf), 2 * C::kTileBytes);
 #pragma unroll
           for (int hf = 0; hf < C::kHalves; ++hf)
             tma_load_4d(sKV + s * C::kTileBytes + hf * C::kAtomBytes, kind ? &tm_v : &tm_k,
-                        bar(C::kBarKVFull + s), 64 * hf, g, 128 * j, b);
+                        bar(C::kBarKVFull + sf), 64 * hf, g, 128 * j, b);
           issued = pos + 1;
         }
       }
       // Every copy this thread started has landed before the CTA can exit (already true on
-      // the normal path; after a consumer gave up this waits, bounded, for copies in flight).
+      // the normal path; after a consumer gave up this waits, bounded, for copies in flight;
+      // a K_j whose V_j was never started leaves its barrier short, and that wait runs out).
       volatile int zero = 0;
       const WaitCtl drain_ctl{&zero, p.timeout_ns};
       mbar_wait(bar(C::kBarQ), 0, drain_ctl);
-      for (int s = 0; s < C::kStages && s < issued; ++s) {
+      for (int s = 0; s < C::kStages && s < issued; s += 2) {
         const int last = s + C::kStages * ((issued - 1 - s) / C::kStages);
         mbar_wait(bar(C::kBarKVFull + s), (last / C::kStages) & 1, drain_ctl);
       }
@@ -390,10 +395,10 @@ __global__ void __launch_bounds__(384, 1)
         }
         return true;
       };
+      // K_j and V_j in shared memory (one barrier for both, at K_j's position).  The MMAs
+      // read them through the async proxy that wrote them; no tcgen05 fence is needed here.
       auto kv_wait = [&](int pos) {
-        const bool ok = mbar_wait(bar(C::kBarKVFull + pos % C::kStages), (pos / C::kStages) & 1, ctl);
-        tc_fence_after();
-        return ok;
+        return mbar_wait(bar(C::kBarKVFull + pos % C::kStages), (pos / C::kStages) & 1, ctl);
       };
       int n[2] = {0, 0};
       bool ok = mbar_wait(bar(C::kBarQ), 0, ctl);
@@ -414,7 +419,6 @@ __global__ void __launch_bounds__(384, 1)
           const int vpos = 2 * kt + 1, kpos = vpos + 1;
           const int vslot = vpos % C::kStages, kslot = kpos % C::kStages;
           const bool nxt = jn < J1;
-          if (!(ok = kv_wait(vpos))) break;
           if (part(0, j)) {
             if (!(ok = issue_pv(0, vslot, j == ts0.first, n[0] & 1))) break;
             ++n[0];
