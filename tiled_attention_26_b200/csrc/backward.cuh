@@ -262,16 +262,15 @@ __global__ void __launch_bounds__(320, 1)
         qt = sb + C::kUOff + (u % C::kUStages) * C::kUnitBytes;
         dot = qt + C::kTileBytes;
       };
+      // (waits on copies into shared memory need no tcgen05 fence: the MMAs read through the
+      // async proxy that wrote them; waits on TMEM written by other warps do)
       bool ok = n_units > 0 && mbar_wait(bar(kBarKV), 0, ctl);
-      tc_fence_after();
       if (ok && (ok = mbar_wait(bar(kBarUFull), 0, ctl))) {
-        tc_fence_after();
         uint32_t qt, dot;
         unit_tiles(0, qt, dot);
         mma_rows(colS, sb + C::kKOff, qt);    // S^T = K Q^T
         tc_commit(bar(kBarS));
         if ((ok = mbar_wait(bar(kBarUDo), 0, ctl))) {
-          tc_fence_after();
           mma_rows(colDP, sb + C::kVOff, dot);  // dP^T = V dO^T
           tc_commit(bar(kBarDP));
         }
@@ -286,7 +285,6 @@ __global__ void __launch_bounds__(320, 1)
         if (nxt) {
           if (!(ok = mbar_wait(bar(kBarUFull + (u + 1) % C::kUStages), ((u + 1) / C::kUStages) & 1, ctl)))
             break;
-          tc_fence_after();
           unit_tiles(u + 1, qn, don);
           mma_rows(colS, sb + C::kKOff, qn);  // S^T of the next unit (after dV read P)
           tc_commit(bar(kBarS));
@@ -298,7 +296,6 @@ __global__ void __launch_bounds__(320, 1)
         if (nxt) {
           if (!(ok = mbar_wait(bar(kBarUDo + (u + 1) % C::kUStages), ((u + 1) / C::kUStages) & 1, ctl)))
             break;
-          tc_fence_after();
           mma_rows(colDP, sb + C::kVOff, don);  // dP^T of the next unit (after dK read dS)
           tc_commit(bar(kBarDP));
         }
@@ -532,18 +529,20 @@ __global__ void __launch_bounds__(320, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(bar(kBarKVFull + s), C::kTileBytes);
+          // K(t) and V(t) land on the full barrier of K(t)'s stage (an even stage)
+          const int sf = (2 * t) % C::kQStages;
+          if (kind == 0) mbar_arrive_expect_tx(bar(kBarKVFull + sf), 2 * C::kTileBytes);
 #pragma unroll
           for (int hf = 0; hf < C::kHalves; ++hf)
             tma_load_4d(sb + C::kQKVOff + s * C::kTileBytes + hf * C::kAtomBytes,
-                        kind ? &tm_v : &tm_k, bar(kBarKVFull + s), 64 * hf, g, 128 * (jlo + t), b);
+                        kind ? &tm_v : &tm_k, bar(kBarKVFull + sf), 64 * hf, g, 128 * (jlo + t), b);
           issued = pos + 1;
         }
       }
       volatile int zero = 0;
       const WaitCtl drain_ctl{&zero, p.timeout_ns};
       mbar_wait(bar(kBarIn), 0, drain_ctl);
-      for (int s = 0; s < C::kQStages && s < issued; ++s) {
+      for (int s = 0; s < C::kQStages && s < issued; s += 2) {
         const int lastp = s + C::kQStages * ((issued - 1 - s) / C::kQStages);
         mbar_wait(bar(kBarKVFull + s), (lastp / C::kQStages) & 1, drain_ctl);
       }
@@ -561,10 +560,10 @@ __global__ void __launch_bounds__(320, 1)
                   idesc_s, kk > 0 ? 1u : 0u);
         }
       };
+      // K(t) and V(t) in shared memory (one barrier for both).  The MMAs read them through
+      // the async proxy that wrote them; no tcgen05 fence is needed after this wait.
       auto kv_wait = [&](int pos) {
-        const bool r = mbar_wait(bar(kBarKVFull + pos % C::kQStages), (pos / C::kQStages) & 1, ctl);
-        tc_fence_after();
-        return r;
+        return mbar_wait(bar(kBarKVFull + pos % C::kQStages), (pos / C::kQStages) & 1, ctl);
       };
       // Order: S(0) dP(0) | S(t+1) dP(t+1) once S(t), dP(t) are in registers | dQ(t) once
       // dS(t) is in TMEM: the next tile's products overlap the elementwise work on this one.
@@ -574,7 +573,6 @@ __global__ void __launch_bounds__(320, 1)
       auto issue_sdp = [&](int t) -> bool {
         if (!kv_wait(2 * t)) return false;
         mma_rows(colS, sb + C::kQOff, tile_addr(2 * t));       // S = Q K^T
-        if (!kv_wait(2 * t + 1)) return false;
         mma_rows(colDP, sb + C::kDOOff, tile_addr(2 * t + 1));  // dP = dO V^T
         tc_commit(bar(kBarSDP));
         tc_commit(bar(kBarKVEmpty + (2 * t + 1) % C::kQStages));  // V(t) is done
