@@ -40,8 +40,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from ncu, keyed by the sha256 of the
 # kernel sources they were taken on; a kernel edited since then reports traffic = null.
 NCU_TRAFFIC = {
-    # profiles/fa_prefill_kernel_mha_causal.md: 532,551,168 B read + 47,900,160 B written
-    "prefill": {"cf0efa0ff3706f95": 580_451_328},
+    # profiles/fa_prefill_kernel_mha_causal.md: 535,730,176 B read + 48,052,736 B written
+    "prefill": {"bb30a856dfed342d": 583_782_912},
     # profiles/fa_decode_split_kernel_decode_int8.md: 1,107,567,616 B read + 6,939,648 B written
     "decode": {"0374b3d7a3500c43": 1_114_507_264},
     # profiles/fa_decode_split_kernel_decode_int8_paged.md: 424,233,984 B read + 4,904,448 B
