@@ -479,6 +479,40 @@ def run_only_backward(args):
     return 0
 
 
+def run_only_decode(args):
+    """fa_decode_int8 on the contiguous decode workload alone, one JSON line (used to profile
+    the decode kernels without the other workloads resident on the device)."""
+    import torch
+
+    import synthetic
+    import tiled_attention_26_b200 as fa
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    w = synthetic.WORKLOADS["decode_int8"]
+    q, k, v, ks, vs = synthetic.make_decode_inputs_torch(w, dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(fa.fa_decode_int8_workspace_bytes(w.B, w.Hq, w.D, w.num_splits),
+                     dtype=torch.uint8, device=dev)
+    ms = time_calls(torch, stream, lambda: fa.fa_decode_int8(q, k, v, ks, vs,
+                                                             num_splits=w.num_splits,
+                                                             scale=w.scale, o=o, lse=lse,
+                                                             workspace=ws, stream=stream),
+                    args.steps, args.warmup)
+    if fa.fa_device_status() != 0:
+        raise RuntimeError("the decode kernels reported a device-side error")
+    nbytes = decode_bytes(w)
+    peaks, _ = load_peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    print(json.dumps({"metric": "INT8 decode GB/s (algorithmic bytes)", "value": gbs,
+                      "unit": "GB/s", "ms_per_call": ms, "bytes_per_call": nbytes,
+                      "steps": args.steps, "warmup": args.warmup,
+                      "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                      "config": {"workload": "decode_int8"}}), flush=True)
+    return 0
+
+
 def run_only_paged(args):
     """fa_decode_int8_paged on the paged workload alone, one JSON line (used to profile the
     paged decode kernels without the other workloads resident on the device)."""
@@ -510,7 +544,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["backward", "prefill", "paged"], default=None,
+    ap.add_argument("--only", choices=["backward", "prefill", "paged", "decode"], default=None,
                     help="time one further row on its own (for profiling); prints its own line")
     args = ap.parse_args()
     if args.impl == "reference":
@@ -521,6 +555,8 @@ def main():
         return run_only_prefill(args)
     if args.only == "paged":
         return run_only_paged(args)
+    if args.only == "decode":
+        return run_only_decode(args)
 
     import torch
 

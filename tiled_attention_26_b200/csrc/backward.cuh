@@ -78,33 +78,40 @@ struct BwdCfg {
 };
 
 // ---------------------------------------------------------------------------------------
-// -D_i = -dO_i . O_i and -L_i * log2(e), one warp per (b, i, h) row (stored negated so the
-// kernels add them); padding rows past Sq get L = +inf and D = 0.  Rows with L = -inf (no
+// -D_i = -dO_i . O_i and -L_i * log2(e) per (b, h, i) row, D / 8 lanes per row (stored negated
+// so the kernels add them); padding rows past Sq get L = +inf and D = 0.  Rows with L = -inf (no
 // visible key) also get +inf: their P is 0.
 // ---------------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdParams p) {
-  const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+  // D / 8 lanes per row, one 16-byte load of O and of dO each (8 bf16); 256 / D rows per warp
+  constexpr int kLanesPerRow = D / 8;
+  constexpr int kRowsPerWarp = 32 / kLanesPerRow;
   const int lane = threadIdx.x & 31;
+  const int sub = lane % kLanesPerRow;
+  const long long row =
+      (static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5)) * kRowsPerWarp +
+      lane / kLanesPerRow;
   const long long rows = static_cast<long long>(p.B) * p.Hq * p.Sq_pad;
-  if (row >= rows) return;
-  const int i = static_cast<int>(row % p.Sq_pad);
-  const long long bh = row / p.Sq_pad;
+  const bool valid = row < rows;  // no early exit: the row's lanes reduce with shuffles
+  const int i = valid ? static_cast<int>(row % p.Sq_pad) : 0;
+  const long long bh = valid ? row / p.Sq_pad : 0;
   const int h = static_cast<int>(bh % p.Hq), b = static_cast<int>(bh / p.Hq);
   float acc = 0.f;
-  if (i < p.Sq) {
-    const size_t base = ((static_cast<size_t>(b) * p.Sq + i) * p.Hq + h) * D;
+  if (valid && i < p.Sq) {
+    const size_t base = ((static_cast<size_t>(b) * p.Sq + i) * p.Hq + h) * D + 8 * sub;
+    const uint4 o4 = __ldg(reinterpret_cast<const uint4*>(p.o + base));
+    const uint4 d4 = __ldg(reinterpret_cast<const uint4*>(p.dout + base));
+    const uint32_t ow[4] = {o4.x, o4.y, o4.z, o4.w}, dw[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
-    for (int e = lane * 2; e < D; e += 64) {
-      const uint32_t o2 = *reinterpret_cast<const uint32_t*>(p.o + base + e);
-      const uint32_t d2 = *reinterpret_cast<const uint32_t*>(p.dout + base + e);
-      acc = fmaf(__uint_as_float(o2 << 16), __uint_as_float(d2 << 16), acc);
-      acc = fmaf(__uint_as_float(o2 & 0xFFFF0000u), __uint_as_float(d2 & 0xFFFF0000u), acc);
+    for (int e = 0; e < 4; ++e) {
+      acc = fmaf(__uint_as_float(ow[e] << 16), __uint_as_float(dw[e] << 16), acc);
+      acc = fmaf(__uint_as_float(ow[e] & 0xFFFF0000u), __uint_as_float(dw[e] & 0xFFFF0000u), acc);
     }
   }
 #pragma unroll
-  for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-  if (lane == 0) {
+  for (int s = kLanesPerRow / 2; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
+  if (valid && sub == 0) {
     float l2 = INFINITY;
     if (i < p.Sq) {
       const float l = p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Sq + i];

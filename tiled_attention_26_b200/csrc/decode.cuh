@@ -151,6 +151,11 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
 __device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
   asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
+// Announce `bytes` of asynchronous copies on `bar` without arriving on it.
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
@@ -314,6 +319,26 @@ __global__ void __launch_bounds__(160, 1) fa_decode_split_kernel(
       const int s = i % C::kStages;
       if (i >= C::kStages && !mbar_wait(bar_empty(s), ((i / C::kStages) - 1) & 1, ctl)) break;
       const int t0 = t_begin + C::kT * i;
+      // The K/V code tiles go first (the bulk of the bytes): their byte count is announced
+      // without an arrival, the copies are issued, and the stage's one arrival comes only after
+      // every lane has registered its scale copies below, so the phase cannot complete early.
+      if (lane == 0) {
+        mbar_expect_tx(bar_full(s), C::kStageBytes);
+        const uint32_t kt = sb + s * C::kStageBytes, vt = kt + C::kTile;
+        for (int t = t0; t < t0 + C::kT; t += box_t) {
+          const uint32_t off = (t - t0) * C::kRow;  // box_t divides kT: stays inside the tile
+          if constexpr (kPaged) {
+            // a box past the split's last key reads the split's last page (its keys are masked)
+            const int pg = page_of(min(t, t_end - 1));
+            const int r0 = t & pmask;
+            tma_load_4d(kt + off, &tm_k, bar_full(s), 0, kvh, r0, pg);
+            tma_load_4d(vt + off, &tm_v, bar_full(s), 0, kvh, r0, pg);
+          } else {
+            tma_load_4d(kt + off, &tm_k, bar_full(s), 0, kvh, t, b);
+            tma_load_4d(vt + off, &tm_v, bar_full(s), 0, kvh, t, b);
+          }
+        }
+      }
       // scales of the stage's keys: 4-byte asynchronous copies, 4 keys per lane
       const uint32_t ks_dst = sb + C::kScaleOff + s * 2 * C::kT * 4;
       const uint32_t vs_dst = ks_dst + C::kT * 4;
@@ -335,25 +360,9 @@ __global__ void __launch_bounds__(160, 1) fa_decode_split_kernel(
           cp_async4(vs_dst + 4 * r, vsrc);
         }
       }
-      cp_async_mbar_arrive(bar_full(s));
+      cp_async_mbar_arrive(bar_full(s));  // each lane: +1 pending now, its arrival on completion
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive_expect_tx(bar_full(s), C::kStageBytes);
-        const uint32_t kt = sb + s * C::kStageBytes, vt = kt + C::kTile;
-        for (int t = t0; t < t0 + C::kT; t += box_t) {
-          const uint32_t off = (t - t0) * C::kRow;  // box_t divides kT: stays inside the tile
-          if constexpr (kPaged) {
-            // a box past the split's last key reads the split's last page (its keys are masked)
-            const int pg = page_of(min(t, t_end - 1));
-            const int r0 = t & pmask;
-            tma_load_4d(kt + off, &tm_k, bar_full(s), 0, kvh, r0, pg);
-            tma_load_4d(vt + off, &tm_v, bar_full(s), 0, kvh, r0, pg);
-          } else {
-            tma_load_4d(kt + off, &tm_k, bar_full(s), 0, kvh, t, b);
-            tma_load_4d(vt + off, &tm_v, bar_full(s), 0, kvh, t, b);
-          }
-        }
-      }
+      if (lane == 0) mbar_arrive(bar_full(s));
       issued = i + 1;
     }
     // Every copy this warp started has landed before the CTA can exit (already true on the

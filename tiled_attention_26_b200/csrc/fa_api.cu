@@ -213,8 +213,10 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
 
   // 1. D and L * log2(e)
   const long long rows = static_cast<long long>(B) * Hq * p.Sq_pad;
-  if ((rows + 7) / 8 > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
-  fa::fa_bwd_prep_kernel<D><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, stream>>>(p);
+  const long long rows_per_block = 8 * (256 / D);  // 8 warps of 256 / D rows each
+  const long long prep_blocks = (rows + rows_per_block - 1) / rows_per_block;
+  if (prep_blocks > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  fa::fa_bwd_prep_kernel<D><<<static_cast<unsigned>(prep_blocks), 256, 0, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
 
   int rc;
