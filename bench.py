@@ -42,11 +42,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC = {
     # profiles/fa_prefill_kernel_mha_causal.md: 535,730,176 B read + 48,052,736 B written
     "prefill": {"bb30a856dfed342d": 583_782_912},
-    # profiles/fa_decode_split_kernel_decode_int8.md: 1,107,567,616 B read + 6,939,648 B written
-    "decode": {"0374b3d7a3500c43": 1_114_507_264},
-    # profiles/fa_decode_split_kernel_decode_int8_paged.md: 424,233,984 B read + 4,904,448 B
+    # profiles/fa_decode_split_kernel_decode_int8.md: 1,107,665,408 B read + 7,308,288 B written
+    "decode": {"5cf4bff363fc9696": 1_114_973_696},
+    # profiles/fa_decode_split_kernel_decode_int8_paged.md: 424,236,032 B read + 4,618,496 B
     # written
-    "paged_decode": {"0374b3d7a3500c43": 429_138_432},
+    "paged_decode": {"5cf4bff363fc9696": 428_854_528},
 }
 
 
