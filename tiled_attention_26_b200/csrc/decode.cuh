@@ -11,8 +11,9 @@
 // heads of that KV head's group).  A producer warp streams the split's keys into a ring of
 // shared-memory stages of 128 keys: the int8 K and V rows by TMA tensor copies (the codes never
 // pass through registers on their way in, so the bytes in flight are bounded by shared memory,
-// not by the register file), their fp32 scales by 4-byte asynchronous copies, all completing on
-// one mbarrier per stage.  Four consumer warps each take 32 keys of every stage, read the rows
+// not by the register file), their fp32 scales by bulk copies (one per page or row segment;
+// 4-byte asynchronous copies when a contiguous scale row is not 16-byte aligned), all
+// completing on one mbarrier per stage.  Four consumer warps each take 32 keys of every stage, read the rows
 // in their MMA fragment layout, convert the codes to fp16 with byte permutes and one fp16
 // subtract, and run both contractions on the tensor cores with mma.sync m16n8k16 (fp32
 // accumulate):
@@ -151,6 +152,15 @@ __device__ __forceinline__ void cp_async4(uint32_t dst, const void* src) {
 __device__ __forceinline__ void cp_async_mbar_arrive(uint32_t bar) {
   asm volatile("cp.async.mbarrier.arrive.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
+// Bulk copy of `bytes` (a multiple of 16, both addresses 16-byte aligned) from global to shared
+// memory, completing on `bar` (no multicast).
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
+                                         uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
 // Announce `bytes` of asynchronous copies on `bar` without arriving on it.
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(bytes)
@@ -223,8 +233,10 @@ __device__ __forceinline__ uint32_t nib_hi16_f16x2(uint32_t biased) {
   return d;
 }
 
+// 3 CTAs per SM for the 8-bit kernels (at most 136 registers a thread): the bytes in flight
+// per SM set the decode's bandwidth.
 template <int D, bool kPaged, int kBits>
-__global__ void __launch_bounds__(160, 1) fa_decode_split_kernel(
+__global__ void __launch_bounds__(160, kBits == 8 ? 3 : 1) fa_decode_split_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const DecodeParams p) {
   using C = DecodeCfg<D, kBits>;
@@ -314,55 +326,73 @@ __global__ void __launch_bounds__(160, 1) fa_decode_split_kernel(
     const float* ks_row = p.k_scale + (static_cast<size_t>(b) * p.Hkv + kvh) * p.Skv;
     const float* vs_row = p.v_scale + (static_cast<size_t>(b) * p.Hkv + kvh) * p.Skv;
 
+    // scales by bulk copies whenever their rows are 16-byte aligned: page scale rows always
+    // are (page_size >= 16); contiguous rows when Skv is a multiple of 4
+    const bool bulk_scales = kPaged || (p.Skv % 4 == 0);
     int issued = 0;
     for (int i = 0; i < n_stages; ++i) {
       const int s = i % C::kStages;
       if (i >= C::kStages && !mbar_wait(bar_empty(s), ((i / C::kStages) - 1) & 1, ctl)) break;
       const int t0 = t_begin + C::kT * i;
-      // The K/V code tiles go first (the bulk of the bytes): their byte count is announced
-      // without an arrival, the copies are issued, and the stage's one arrival comes only after
-      // every lane has registered its scale copies below, so the phase cannot complete early.
-      if (lane == 0) {
-        mbar_expect_tx(bar_full(s), C::kStageBytes);
-        const uint32_t kt = sb + s * C::kStageBytes, vt = kt + C::kTile;
-        for (int t = t0; t < t0 + C::kT; t += box_t) {
-          const uint32_t off = (t - t0) * C::kRow;  // box_t divides kT: stays inside the tile
-          if constexpr (kPaged) {
-            // a box past the split's last key reads the split's last page (its keys are masked)
-            const int pg = page_of(min(t, t_end - 1));
-            const int r0 = t & pmask;
-            tma_load_4d(kt + off, &tm_k, bar_full(s), 0, kvh, r0, pg);
-            tma_load_4d(vt + off, &tm_v, bar_full(s), 0, kvh, r0, pg);
-          } else {
+      const uint32_t ks_dst = sb + C::kScaleOff + s * 2 * C::kT * 4;
+      const uint32_t vs_dst = ks_dst + C::kT * 4;
+      if (bulk_scales) {
+        // One thread issues everything: the K/V code boxes and, beside each, its keys' scales
+        // as one bulk copy (a page's scales are contiguous; so are a row segment's).  Keys past
+        // the split's end get real scales of the same page or row; the consumers mask them.
+        if (lane == 0) {
+          const uint32_t seg =
+              kPaged ? C::kT * 4 : static_cast<uint32_t>(min(C::kT, p.Skv - t0)) * 4;
+          mbar_arrive_expect_tx(bar_full(s), C::kStageBytes + 2 * seg);
+          const uint32_t kt = sb + s * C::kStageBytes, vt = kt + C::kTile;
+          for (int t = t0; t < t0 + C::kT; t += box_t) {
+            const uint32_t off = (t - t0) * C::kRow;  // box_t divides kT: stays inside the tile
+            if constexpr (kPaged) {
+              // a box past the split's last key reads the split's last page
+              const int pg = page_of(min(t, t_end - 1));
+              const int r0 = t & pmask;
+              tma_load_4d(kt + off, &tm_k, bar_full(s), 0, kvh, r0, pg);
+              tma_load_4d(vt + off, &tm_v, bar_full(s), 0, kvh, r0, pg);
+              const size_t idx = ((static_cast<size_t>(pg) * p.Hkv + kvh) << p.page_shift) + r0;
+              bulk_g2s(ks_dst + 4 * (t - t0), p.k_scale + idx, 4 * box_t, bar_full(s));
+              bulk_g2s(vs_dst + 4 * (t - t0), p.v_scale + idx, 4 * box_t, bar_full(s));
+            } else {
+              tma_load_4d(kt + off, &tm_k, bar_full(s), 0, kvh, t, b);
+              tma_load_4d(vt + off, &tm_v, bar_full(s), 0, kvh, t, b);
+            }
+          }
+          if constexpr (!kPaged) {
+            bulk_g2s(ks_dst, ks_row + t0, seg, bar_full(s));
+            bulk_g2s(vs_dst, vs_row + t0, seg, bar_full(s));
+          }
+        }
+        __syncwarp();
+      } else {
+        // Contiguous scale rows that are not 16-byte aligned: 4-byte asynchronous copies, 4 keys
+        // per lane.  The K/V code tiles still go first: their byte count is announced without
+        // an arrival, and the stage's one arrival comes only after every lane has registered
+        // its scale copies, so the phase cannot complete early.
+        if (lane == 0) {
+          mbar_expect_tx(bar_full(s), C::kStageBytes);
+          const uint32_t kt = sb + s * C::kStageBytes, vt = kt + C::kTile;
+          for (int t = t0; t < t0 + C::kT; t += box_t) {
+            const uint32_t off = (t - t0) * C::kRow;
             tma_load_4d(kt + off, &tm_k, bar_full(s), 0, kvh, t, b);
             tma_load_4d(vt + off, &tm_v, bar_full(s), 0, kvh, t, b);
           }
         }
-      }
-      // scales of the stage's keys: 4-byte asynchronous copies, 4 keys per lane
-      const uint32_t ks_dst = sb + C::kScaleOff + s * 2 * C::kT * 4;
-      const uint32_t vs_dst = ks_dst + C::kT * 4;
 #pragma unroll
-      for (int j = 0; j < C::kT / 32; ++j) {
-        const int r = lane + 32 * j, t = t0 + r;
-        if (t < t_end) {
-          const float *ksrc, *vsrc;
-          if constexpr (kPaged) {
-            const size_t idx =
-                ((static_cast<size_t>(page_of(t)) * p.Hkv + kvh) << p.page_shift) + (t & pmask);
-            ksrc = p.k_scale + idx;
-            vsrc = p.v_scale + idx;
-          } else {
-            ksrc = ks_row + t;
-            vsrc = vs_row + t;
+        for (int j = 0; j < C::kT / 32; ++j) {
+          const int r = lane + 32 * j, t = t0 + r;
+          if (t < t_end) {
+            cp_async4(ks_dst + 4 * r, ks_row + t);
+            cp_async4(vs_dst + 4 * r, vs_row + t);
           }
-          cp_async4(ks_dst + 4 * r, ksrc);
-          cp_async4(vs_dst + 4 * r, vsrc);
         }
+        cp_async_mbar_arrive(bar_full(s));  // each lane: +1 pending now, its arrival on completion
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_full(s));
       }
-      cp_async_mbar_arrive(bar_full(s));  // each lane: +1 pending now, its arrival on completion
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_full(s));
       issued = i + 1;
     }
     // Every copy this warp started has landed before the CTA can exit (already true on the
