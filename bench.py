@@ -513,6 +513,28 @@ def run_only_decode(args):
     return 0
 
 
+def run_only_int4(args):
+    """fa_decode_int4 on the INT4 decode workload alone, one JSON line (used to profile the
+    4-bit decode kernels without the other workloads resident on the device)."""
+    import torch
+
+    import synthetic
+    import tiled_attention_26_b200 as fa
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    ms, nbytes = measure_int4_decode(fa, synthetic, torch, dev, stream, steps=args.steps,
+                                     warmup=args.warmup)
+    peaks, _ = load_peaks()
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    print(json.dumps({"metric": "INT4 decode GB/s (algorithmic bytes)", "value": gbs,
+                      "unit": "GB/s", "ms_per_call": ms, "bytes_per_call": nbytes,
+                      "steps": args.steps, "warmup": args.warmup,
+                      "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                      "config": {"workload": "decode_int4"}}), flush=True)
+    return 0
+
+
 def run_only_paged(args):
     """fa_decode_int8_paged on the paged workload alone, one JSON line (used to profile the
     paged decode kernels without the other workloads resident on the device)."""
@@ -544,7 +566,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["backward", "prefill", "paged", "decode"], default=None,
+    ap.add_argument("--only", choices=["backward", "prefill", "paged", "decode", "int4"],
+                    default=None,
                     help="time one further row on its own (for profiling); prints its own line")
     args = ap.parse_args()
     if args.impl == "reference":
@@ -557,6 +580,8 @@ def main():
         return run_only_paged(args)
     if args.only == "decode":
         return run_only_decode(args)
+    if args.only == "int4":
+        return run_only_int4(args)
 
     import torch
 
