@@ -216,18 +216,20 @@ __device__ __forceinline__ uint32_t swz(uint32_t off) {
   else return off;
 }
 
-// INT4 codes of an offset-binary word (code + 8 per nibble) -> fp16x2, exactly.  In fp16 with
-// exponent 2^10 the mantissa counts units, so: nibbles at bits [0,4) and [16,20) give 1024 + n,
-// minus 1032 leaves n - 8; nibbles at bits [4,8) and [20,24) give 1024 + 16 n, minus 1152
-// leaves 16 (n - 8), scaled by 16 (the caller folds 1/16 into the other operand or the output).
-__device__ __forceinline__ uint32_t nib_lo_f16x2(uint32_t biased) {
-  const uint32_t h = (biased & 0x000F000Fu) | 0x64006400u;
+// INT4 codes (4-bit two's complement) of a word -> fp16x2, exactly.  Flipping the top bit of a
+// nibble gives its offset-binary value n = code + 8; the flip rides in the magic constant, so
+// one logic op both masks and biases.  In fp16 with exponent 2^10 the mantissa counts units:
+// nibbles at bits [0,4) and [16,20) give 1024 + n, minus 1032 leaves the code; nibbles at bits
+// [4,8) and [20,24) give 1024 + 16 n, minus 1152 leaves 16 x the code (the caller folds 1/16
+// into the other operand or the output).
+__device__ __forceinline__ uint32_t nib_lo_f16x2(uint32_t raw) {
+  const uint32_t h = (raw & 0x000F000Fu) ^ 0x64086408u;
   uint32_t d;
   asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(h), "r"(0x64086408u));
   return d;
 }
-__device__ __forceinline__ uint32_t nib_hi16_f16x2(uint32_t biased) {
-  const uint32_t h = (biased & 0x00F000F0u) | 0x64006400u;
+__device__ __forceinline__ uint32_t nib_hi16_f16x2(uint32_t raw) {
+  const uint32_t h = (raw & 0x00F000F0u) ^ 0x64806480u;
   uint32_t d;
   asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(h), "r"(0x64806480u));
   return d;
@@ -247,7 +249,9 @@ __global__ void __launch_bounds__(160, kBits == 8 ? 3 : 1) fa_decode_split_kerne
   constexpr int DPT = D / 8;            // PV: output dims of one thread
   constexpr int VB = DPT * kBits / 8;   // ... as bytes of each V row
   constexpr int VW = (VB + 3) / 4;      // ... as 32-bit words
-  constexpr uint32_t kBias = kBits == 8 ? 0x80808080u : 0x88888888u;  // to offset binary
+  // INT8 codes go to offset binary on load (the byte permutes need it); INT4 nibbles are biased
+  // inside their conversion
+  constexpr uint32_t kBias = kBits == 8 ? 0x80808080u : 0u;
   // the merge kernel may be scheduled as soon as every CTA of this grid has started
   asm volatile("griddepcontrol.launch_dependents;");
 
@@ -625,10 +629,10 @@ __global__ void __launch_bounds__(160, kBits == 8 ? 3 : 1) fa_decode_split_kerne
             a3 = codes_to_f16x2(x89, kSelB23);
           } else {
             const int w = mt >> 2;
-            const uint32_t sel = (mt & 2) ? 0x7632u : 0x5410u;
-            // [k0.b, k0.b', k1.b, k1.b'], shifted so that this m-tile's byte is the low one
-            const uint32_t x01 = prmt(r[0][w], r[1][w], sel) >> (8 * (mt & 1));
-            const uint32_t x89 = prmt(r[2][w], r[3][w], sel) >> (8 * (mt & 1));
+            // byte mt & 3 of the first key's word into byte 0, of the second key's into byte 2
+            constexpr uint32_t kSel[4] = {0x4400u, 0x5511u, 0x6622u, 0x7733u};
+            const uint32_t x01 = prmt(r[0][w], r[1][w], kSel[mt & 3]);  // keys 2c, 2c+1
+            const uint32_t x89 = prmt(r[2][w], r[3][w], kSel[mt & 3]);  // keys 2c+8, 2c+9
             // dim 2mt (low nibble) as is; dim 2mt+1 (high nibble) times 16, undone at the end
             a0 = nib_lo_f16x2(x01);
             a1 = nib_hi16_f16x2(x01);
