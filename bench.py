@@ -42,11 +42,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC = {
     # profiles/fa_prefill_kernel_mha_causal.md: 535,730,176 B read + 48,052,736 B written
     "prefill": {"bb30a856dfed342d": 583_782_912},
-    # profiles/fa_decode_split_kernel_decode_int8.md: 1,107,921,664 B read + 10,537,984 B written
-    "decode": {"0bd6521c8686c98c": 1_118_459_648},
-    # profiles/fa_decode_split_kernel_decode_int8_paged.md: 424,312,064 B read + 4,839,680 B
+    # profiles/fa_decode_split_kernel_decode_int8.md: 1,107,942,400 B read + 10,583,808 B written
+    "decode": {"a06a790a147221ec": 1_118_526_208},
+    # profiles/fa_decode_split_kernel_decode_int8_paged.md: 424,260,352 B read + 4,880,128 B
     # written
-    "paged_decode": {"0bd6521c8686c98c": 429_151_744},
+    "paged_decode": {"a06a790a147221ec": 429_140_480},
 }
 
 
