@@ -10,7 +10,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libfa.so")
 SOURCES = [os.path.join(CSRC, "fa_api.cu")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("sm100.cuh", "prefill.cuh", "decode.cuh")] + [
+DEPS = SOURCES + sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")) + [
     os.path.join(ROOT, "include", "fa.h")]
 
 NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
