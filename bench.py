@@ -7,14 +7,22 @@ One step = one pass of the whole path over one batch of synthetic input:
   * decode   (fa_decode_int8, split kernel + combine kernel): B=16, Hq=32, Hkv=8, Skv=32768,
     D=128, INT8 KV cache with per-token scales, 16 splits (KV-read GB/s).
 After the timed steps, short loops of their own time the paged, variable-length decode
-(fa_decode_int8_paged, "paged_decode") and the INT4 decode (fa_decode_int4, "int4_decode");
-they are not part of the step.
+(fa_decode_int8_paged, "paged_decode"), the INT4 decode (fa_decode_int4, "int4_decode"), the
+masked and global+local forward passes, the backward pass, and the GQA causal, GQA
+sliding-window and MQA causal forward workloads ("gqa_causal", "gqa_sw512", "mqa_causal"); they
+are not part of the step.  Tensor-core fractions divide by the measured burst bf16 peak unless
+the clock samples of the timed region saw the power cap.
 Inputs are seeded synthetic N(0,1) draws (see synthetic.py) resident in HBM; both inputs are
 larger than the 126 MB L2 (prefill 268 MB, decode 1.1 GB), so no flush is needed between steps.
 
 Prints ONE JSON line (rank 0).  Under torchrun every rank runs the same workload on its own
 GPU with its own seeds (independent problems, weak scaling, no data-path collective); times are
 CUDA-event times, max over ranks.
+
+On rank 0 of a one-GPU run the fp64 CPU oracle is also timed on bounded samples of the
+prefill and decode workloads ("cpu_baseline", "cpu_baseline_decode"), and the INT8 / INT4 decode
+results of the first two sequences are compared with the oracle over the unquantised bf16 K and
+V ("kv_quant_error", informational).
 
 ``--impl reference`` times the fp64 CPU oracle on a bounded row sample of the same prefill
 workload instead (rank 0 only).
@@ -48,6 +56,11 @@ NCU_TRAFFIC = {
     # written
     "paged_decode": {"a06a790a147221ec": 429_140_480},
 }
+
+
+# the kernel that runs the plain prefill (causal / window / full) and its sources
+KERNEL_PREFILL = "fa_prefill_kernel<{D}>"
+PREFILL_SOURCES = ("prefill.cuh", "sm100.cuh")
 
 
 def source_hash(*names):
@@ -124,6 +137,58 @@ def global_local_flops(w, n_global: int) -> int:
     extra = np.maximum(0, np.minimum(n_global, lo) - 0)
     pairs = np.where(i < n_global, w.Skv, band + extra)
     return int(pairs.sum()) * 4 * w.D * w.B * w.Hq
+
+
+def tile_ceiling(w) -> float:
+    """Useful fraction of the score-tile area the prefill kernel computes for workload w: visible
+    (query, key) pairs over (tiles computed x 128 x 128).  A Q tile holds 128 rows = 128 / Gp
+    tokens x Gp query heads of one KV group (Gp the largest power of two <= 8 dividing Hq/Hkv);
+    it computes every 128-key tile that holds a key one of its rows sees."""
+    G = w.Hq // w.Hkv
+    gp = 1
+    while gp < 8 and G % (2 * gp) == 0:
+        gp *= 2
+    tpt = 128 // gp
+    off = w.Skv - w.Sq
+    tiles = 0
+    for t0 in range(0, w.Sq, tpt):
+        t1 = min(t0 + tpt, w.Sq) - 1
+        hi = min(t1 + off, w.Skv - 1) if w.causal else w.Skv - 1
+        lo = max(0, t0 + off - w.window + 1) if w.window > 0 else 0
+        if hi >= lo and hi >= 0:
+            tiles += hi // 128 - lo // 128 + 1
+    computed = tiles * (w.Hq // gp) * w.B * 128 * 128
+    return prefill_flops(w) / (4 * w.D) / computed
+
+
+def tensor_peak(peaks, clk):
+    """The dense bf16 peak a prefill kernel is held against: the burst figure, unless the clock
+    samples of the timed region saw the power cap, then the sustained one."""
+    if "sw_power_cap" in (clk or {}).get("reasons", []):
+        return peaks["bf16_tflops_sustained"], "sustained (sw_power_cap seen in the timed region)"
+    return peaks["bf16_tflops"], "burst (no power cap seen in the timed region)"
+
+
+def measure_prefill_configs(fa, synthetic, torch, dev, stream, steps: int, warmup: int,
+                            seed_off: int = 0):
+    """fa_fwd on the GQA causal, GQA sliding-window and MQA causal workloads, each in its own
+    loop.  Returns {name: (ms per call, algorithmic flops)}."""
+    out = {}
+    for name in ("gqa_causal", "gqa_sw512", "mqa_causal"):
+        w = synthetic.WORKLOADS[name]
+        q = synthetic.normal_bf16_torch(w.seed(0) + seed_off, w.q_shape(), dev)
+        k = synthetic.normal_bf16_torch(w.seed(1) + seed_off, w.kv_shape(), dev)
+        v = synthetic.normal_bf16_torch(w.seed(2) + seed_off, w.kv_shape(), dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=dev)
+        ms = time_calls(torch, stream, lambda: fa.fa_fwd(q, k, v, causal=w.causal, window=w.window,
+                                                          scale=w.scale, o=o, lse=lse,
+                                                          stream=stream), steps, warmup)
+        out[name] = (ms, prefill_flops(w))
+        del q, k, v, o, lse
+    if fa.fa_device_status() != 0:
+        raise RuntimeError("a prefill kernel reported a device-side error")
+    return out
 
 
 def measure_mask_variants(fa, synthetic, torch, dev, stream, steps: int, warmup: int):
@@ -341,6 +406,77 @@ def cpu_baseline(w, budget_s: float, seed: int):
                       f"fp64, {dt:.1f} s"}, dt
 
 
+def cpu_baseline_decode(dev_inputs, w, budget_s: float, seed: int):
+    """The fp64 oracle's INT8 decode (as it stands) on a bounded sample of (b, h) rows of the
+    decode workload, on the host cores: algorithmic bytes of the sampled rows per second."""
+    import numpy as np
+
+    import oracle
+    q, kq, vq, ks, vs = (t.cpu().numpy() for t in dev_inputs)
+    q = q.view(np.uint16) if q.dtype != np.uint16 else q
+    G = w.Hq // w.Hkv
+
+    def rows(n, s):
+        import synthetic
+        raw = synthetic.splitmix64(s, 0, 2 * n).reshape(-1, 2)
+        return np.stack([raw[:, 0] % np.uint64(w.B), raw[:, 1] % np.uint64(w.Hq)],
+                        axis=1).astype(np.int64)
+
+    def bytes_of(r):
+        # each row reads its KV head's codes and scales once (the kernel reads them once per
+        # group of G rows), plus its q, o and LSE
+        per_kv = 2 * w.Skv * w.D + 2 * w.Skv * 4
+        return len(r) * (per_kv / G + 2 * w.D * 2 + 4)
+
+    t0 = time.perf_counter()
+    oracle.decode_int8_rows(q, kq, vq, ks, vs, w.scale, 1, rows(8, seed))
+    per_row = max((time.perf_counter() - t0) / 8, 1e-4)
+    r = rows(max(8, int(budget_s / per_row)), seed + 1)
+    t0 = time.perf_counter()
+    oracle.decode_int8_rows(q, kq, vq, ks, vs, w.scale, 1, r)
+    dt = time.perf_counter() - t0
+    return {"value": bytes_of(r) / dt / 1e9, "unit": "GB/s", "cores": oracle.max_threads(),
+            "kind": "oracle",
+            "sample": f"{len(r)} seeded (b, h) rows of the INT8 decode workload, all "
+                      f"{w.Skv} keys each, fp64, {dt:.1f} s (bytes counted as the kernel reads "
+                      f"them: each KV head's codes and scales once per {G} query heads)"}
+
+
+def kv_quant_error(fa, synthetic, torch, dev, w, n_batch: int = 2):
+    """Informational: how far INT8 and INT4 KV-cache decode land from attention over the
+    unquantised bf16 K and V, on the first n_batch sequences of the decode workload (the same
+    seeded bf16 values the INT8 cache was quantised from).  The reference is the fp64 oracle
+    over the bf16 values; the quantised results are this library's decode kernels."""
+    import numpy as np
+
+    import oracle
+    shp = (n_batch, w.Skv, w.Hkv, w.D)
+    q = synthetic.normal_bf16_torch(w.seed(0), (n_batch, 1, w.Hq, w.D), dev)
+    k = synthetic.normal_bf16_torch(w.seed(1), shp, dev)
+    v = synthetic.normal_bf16_torch(w.seed(2), shp, dev)
+    host = [t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16) for t in (q, k, v)]
+    o_ref, _ = oracle.attn(host[0], host[1], host[2], w.scale, 0, 0)
+    o_ref = o_ref.reshape(n_batch, w.Hq, w.D)
+    out = {}
+    for name, quant, call in (("int8", synthetic.quantize_int8_per_token_torch, fa.fa_decode_int8),
+                              ("int4", synthetic.quantize_int4_per_token_torch, fa.fa_decode_int4)):
+        kq, ks = quant(k)
+        vq, vs = quant(v)
+        o, _ = call(q, kq, vq, ks, vs, num_splits=w.num_splits, scale=w.scale)
+        got = o.float().cpu().numpy().astype(np.float64).reshape(n_batch, w.Hq, w.D)
+        d = np.abs(got - o_ref)
+        out[name] = {"max_abs": float(d.max()), "mean_abs": float(d.mean()),
+                     "rel_l2": float(np.linalg.norm(d) / np.linalg.norm(o_ref)),
+                     "max_abs_over_max_ref": float(d.max() / np.abs(o_ref).max())}
+    if fa.fa_device_status() != 0:
+        raise RuntimeError("a decode kernel reported a device-side error")
+    return {"rows": f"{n_batch} x {w.Hq} (b, h) rows of the INT8 decode workload, {w.Skv} keys",
+            "reference": "fp64 oracle over the unquantised bf16 K and V",
+            "pages_claim": "precision loss < 0.5 % with the INT8 KV cache (no metric stated); "
+                           "rel_l2 is the closest figure here",
+            **out}
+
+
 def run_reference(args):
     import synthetic
 
@@ -473,7 +609,7 @@ def run_only_backward(args):
     print(json.dumps({"metric": "attention backward TFLOP/s (10*D flops per visible pair)",
                       "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                       "ms_per_call": ms, "steps": args.steps, "warmup": args.warmup,
-                      "frac": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"],
+                      "frac_of_burst": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
                       "config": {"workload": "mha_causal (B=2, H=32, S=4096, D=128, causal)"}}),
           flush=True)
     return 0
@@ -680,6 +816,9 @@ def main():
     bw_ms, bw_flops = measure_backward(fa, synthetic, torch, dev, stream, steps=min(K, 50),
                                        warmup=max(3, args.warmup // 4))
     bw_ms = max_over_ranks(bw_ms)
+    pc = measure_prefill_configs(fa, synthetic, torch, dev, stream, steps=min(K, 100),
+                                 warmup=max(3, args.warmup // 4), seed_off=seed_off)
+    pc = {kk: (max_over_ranks(ms), fl) for kk, (ms, fl) in pc.items()}
 
     # ---- end to end through the public API, host buffers, copies inside the timed region ----
     e2e = None
@@ -718,12 +857,25 @@ def main():
                           "unit": "GB/s"},
                "ms_per_step": (p_ms + d_ms) / E}
 
-    cpu = None
+    cpu = cpu_dec = qerr = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu, _ = cpu_baseline(wp, args.cpu_budget, seed=wp.seed(40))
+        cpu_dec = cpu_baseline_decode((dq, dk, dv, dks, dvs), wd, args.cpu_budget,
+                                      seed=wd.seed(40))
+        qerr = kv_quant_error(fa, synthetic, torch, dev, wd)
+
+    tpeak, tpeak_src = tensor_peak(peaks, clk)
+
+    def prefill_row(name, desc):
+        ms, fl = pc[name]
+        w = synthetic.WORKLOADS[name]
+        tf = fl / (ms * 1e-3) / 1e12
+        return {"workload": desc, "kernel": KERNEL_PREFILL.format(D=w.D), "ms_per_call": ms,
+                "flops_per_call": fl, "achieved": tf, "unit": "TFLOP/s", "peak": tpeak,
+                "frac": tf / tpeak, "tile_ceiling": tile_ceiling(w)}
 
     if rank == 0:
-        tp = NCU_TRAFFIC["prefill"].get(source_hash("prefill.cuh", "sm100.cuh"))
+        tp = NCU_TRAFFIC["prefill"].get(source_hash(*PREFILL_SOURCES))
         td = NCU_TRAFFIC["decode"].get(source_hash("decode.cuh", "sm100.cuh"))
         line = {
             "metric": METRIC,
@@ -749,16 +901,16 @@ def main():
             },
             "decode": {"value": dec_gbs, "unit": "GB/s", "frac_of_hbm": dec_gbs / world / peaks["hbm_gbs"],
                        "ms_per_call": dec_sum / K},
-            # The prefill kernel is timed inside a long back-to-back loop of steps under the
-            # power cap, so its denominator is the sustained dense bf16 figure; the burst
-            # figure's fraction is reported beside it.
+            # The denominator is the burst dense bf16 figure unless the clock samples of the
+            # timed region saw the power cap (then the sustained one); the fraction of the
+            # other figure is reported beside it.
             "roofline": {"bound": "tensor", "achieved": achieved,
-                         "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                         "frac": achieved / peaks["bf16_tflops_sustained"],
+                         "peak": tpeak, "unit": "TFLOP/s",
+                         "frac": achieved / tpeak,
                          "frac_of_burst_peak": achieved / peaks["bf16_tflops"],
-                         "traffic": tp, "kernel": "fa_prefill_kernel<128>",
-                         "peak_source": f"{peak_src} bf16 dense, sustained (burst "
-                                        f"{peaks['bf16_tflops']:.1f})",
+                         "frac_of_sustained_peak": achieved / peaks["bf16_tflops_sustained"],
+                         "traffic": tp, "kernel": KERNEL_PREFILL.format(D=wp.D),
+                         "peak_source": f"{peak_src} bf16 dense, {tpeak_src}",
                          "ms_per_launch": pre_avg_s * 1e3},
             "roofline_decode": {"bound": "hbm", "achieved": d_achieved, "peak": peaks["hbm_gbs"],
                                 "unit": "GB/s", "frac": d_achieved / peaks["hbm_gbs"],
@@ -789,23 +941,30 @@ def main():
                             "fp32 bias mask [1, 32, 4096, 4096]",
                 "kernel": "fa_prefill_kernel<128, mask>", "ms_per_call": mv["masked"][0],
                 "achieved": mv["masked"][1] / (mv["masked"][0] * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "frac": mv["masked"][1] / (mv["masked"][0] * 1e-3) / 1e12
-                        / peaks["bf16_tflops_sustained"]},
+                "frac": mv["masked"][1] / (mv["masked"][0] * 1e-3) / 1e12 / tpeak},
             "global_local_prefill": {
-                "workload": "gqa_sw512 (B=3, Hq=32, Hkv=8, S=4096, D=128, causal window 512) + "
+                "workload": "gqa_sw512 (B=1, Hq=32, Hkv=8, S=4096, D=128, causal window 512) + "
                             "64 global tokens",
                 "kernel": "fa_prefill_kernel<128, global>", "ms_per_call": mv["global_local"][0],
                 "achieved": mv["global_local"][1] / (mv["global_local"][0] * 1e-3) / 1e12,
                 "unit": "TFLOP/s",
-                "frac": mv["global_local"][1] / (mv["global_local"][0] * 1e-3) / 1e12
-                        / peaks["bf16_tflops_sustained"]},
+                "frac": mv["global_local"][1] / (mv["global_local"][0] * 1e-3) / 1e12 / tpeak},
             "backward": {
                 "workload": "mha_causal (B=2, H=32, S=4096, D=128, causal): fa_bwd after fa_fwd",
                 "kernels": "fa_bwd_prep_kernel + fa_bwd_dkdv_kernel<128> + fa_bwd_dq_kernel<128>",
                 "ms_per_call": bw_ms, "flops_per_call": bw_flops,
                 "achieved": bw_flops / (bw_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "frac": bw_flops / (bw_ms * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]},
+                "frac": bw_flops / (bw_ms * 1e-3) / 1e12 / tpeak},
+            "gqa_causal": prefill_row("gqa_causal", "GQA causal (B=1, Hq=32, Hkv=8, S=4096, "
+                                                    "D=128)"),
+            "gqa_sw512": prefill_row("gqa_sw512", "GQA causal, sliding window W=512 (B=1, Hq=32, "
+                                                  "Hkv=8, S=4096, D=128); tile_ceiling = visible "
+                                                  "pairs / computed tile area"),
+            "mqa_causal": prefill_row("mqa_causal", "MQA causal (B=1, Hq=232, Hkv=1, S=2048, "
+                                                    "D=64)"),
             "cpu_baseline": cpu,
+            "cpu_baseline_decode": cpu_dec,
+            "kv_quant_error": qerr,
             "e2e": e2e,
             "gpu_launches": 3 * K,
             "clocks": clk,

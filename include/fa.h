@@ -26,16 +26,22 @@
  *
  * Conventions shared by every entry point
  *   - All tensor arguments are DEVICE pointers owned by the caller, contiguous, 16-byte
- *     aligned.  The library allocates no device memory in these calls and keeps only host-side
- *     state (resolved driver entry points and per-device kernel attributes).
+ *     aligned.  The library allocates no device memory in these calls.  Besides host-side
+ *     state (resolved driver entry points and per-device kernel attributes) it holds two kinds
+ *     of static device data, reserved when the module loads on a device: a 4-byte status word
+ *     (see fa_device_status) and the FA_DECODE_INT8_NOALLOC_MAX_SCRATCH-byte scratch array of
+ *     fa_decode_int8_noalloc, which every GPU that loads the library holds until exit, even if
+ *     only other entry points are called there.
  *   - bf16 tensors are raw IEEE bfloat16 bit patterns; fp32 tensors are IEEE binary32.
  *   - Calls validate their arguments synchronously and enqueue their kernels asynchronously on
  *     `stream` (a cudaStream_t; NULL is the legacy default stream).  Errors that happen on the
  *     device surface at the caller's next synchronisation; fa_device_status() reports the
  *     library's own device-side failures (a bounded wait that gave up, an out-of-range index
  *     read from device memory).
- *   - Thread safety: calls may be made from several host threads; they share no mutable
- *     state beyond one-time initialisation, which is guarded.
+ *   - Thread safety: calls may be made from several host threads.  Their only shared mutable
+ *     state is the guarded one-time initialisation, the per-device status word, and the
+ *     scratch array of fa_decode_int8_noalloc (see there: calls of that function that overlap
+ *     on the GPU race on it).
  */
 #ifndef FA_H_
 #define FA_H_
@@ -173,7 +179,12 @@ FA_API int fa_decode_int8(const void* q, const int8_t* k, const int8_t* v, const
  * cudaMalloc, cudaFree or other allocating routine.
  *
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
- * that device current and caches it; make that first call before any stream capture.
+ * that device current and caches it.  If no other fa_* call has launched a kernel on that device
+ * yet, that lookup is also what loads the library's module there (CUDA loads modules lazily),
+ * and loading the module reserves the array and the kernels' code: an implicit allocation that
+ * may synchronise the device.  Callers for whom that matters make one call of this function (or
+ * of any fa_* entry point that launches a kernel) on each device at set-up time, before any
+ * stream capture and before the latency-critical or allocation-free part of their program.
  *
  * Every call on a GPU shares the one array, and the array keeps the last call's contents (the
  * kernels overwrite every byte they read, so nothing needs clearing).  Calls whose kernels can
@@ -256,11 +267,17 @@ FA_API int fa_decode_int4_paged(const void* q, const uint8_t* k_pages, const uin
 FA_API const char* fa_status_string(int status);
 
 /*
- * Synchronises `stream`, then reads and clears the library's device status word on the current
- * device.  Returns FA_ERR_TIMEOUT if a kernel launched by this library gave up a bounded wait
+ * Takes the library's device status word on the current device: a one-thread kernel on
+ * `stream` swaps it with 0 in one atomic operation, so a bit that a running kernel sets is
+ * never lost between the read and the clear; then `stream` is synchronised and the old value
+ * read back.  Returns FA_ERR_TIMEOUT if a kernel launched by this library gave up a bounded wait
  * since the last call, else FA_ERR_DEVICE_INDEX if a kernel met an out-of-range page id or
- * sequence length (the outputs of such a call are undefined), FA_ERR_CUDA if the
- * synchronisation failed, else FA_OK.
+ * sequence length (the outputs of such a call are undefined), FA_ERR_CUDA if a CUDA call
+ * failed, else FA_OK.
+ * The word is one per device and process, not per stream: it collects the reports of every
+ * kernel of this library on that device, whatever stream launched it, and a call consumes
+ * them all.  Callers that run several streams should call it after synchronising all of them.
+ * Concurrent calls from several host threads are serialised by the library.
  */
 FA_API int fa_device_status(void* stream);
 

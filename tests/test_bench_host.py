@@ -78,3 +78,27 @@ def test_weak_scaling_throughput():
     # 4 ranks, 10 steps of 3e9 units each, slowest rank 20 ms: 4 * 10 * 3e9 / 0.02 s
     assert bench.weak_scaling_throughput(4, 10, 3e9, 20.0) == 4 * 10 * 3e9 / 0.02
     assert bench.weak_scaling_throughput(1, 1, 1.0, 1.0) == 1000.0
+
+
+def test_tile_ceiling_against_a_tile_by_tile_count():
+    """The useful fraction of the computed score-tile area: for the sliding window of 512 keys
+    the page's workload gives 5 key tiles of 128 per 128-row Q tile against 512 x 128 useful
+    pairs (80 %, up to the first rows); a non-causal square problem wastes nothing."""
+    w = synthetic.WORKLOADS["gqa_sw512"]
+    assert abs(bench.tile_ceiling(w) - 0.8) < 2e-3
+    assert bench.tile_ceiling(synthetic.WORKLOADS["tiny"]) == 1.0
+    # brute force on a small causal MQA-like shape: 8 heads packed per tile (16 tokens)
+    small = synthetic.Workload("t", 0, 1, 8, 1, 100, 100, 64, 1)
+    tiles = 0
+    for t0 in range(0, 100, 16):
+        hi = min(t0 + 15, 99)
+        tiles += hi // 128 + 1
+    useful = _pairs_brute(100, 100, 1, 0) * 8
+    assert abs(bench.tile_ceiling(small) - useful / (tiles * 128 * 128)) < 1e-12
+
+
+def test_tensor_peak_follows_the_power_cap_samples():
+    peaks = {"bf16_tflops": 1629.0, "bf16_tflops_sustained": 1374.6, "hbm_gbs": 6557.4}
+    assert bench.tensor_peak(peaks, {"reasons": []})[0] == 1629.0
+    assert bench.tensor_peak(peaks, {"reasons": ["sw_power_cap"]})[0] == 1374.6
+    assert bench.tensor_peak(peaks, None)[0] == 1629.0

@@ -41,10 +41,6 @@ struct BwdParams {
   uint64_t timeout_ns;
 };
 
-#ifndef FA_BWD_KEY_TILE_MAJOR
-#define FA_BWD_KEY_TILE_MAJOR 1
-#endif
-
 template <int D>
 struct BwdCfg {
   static constexpr int kThreads = 320;
@@ -158,16 +154,10 @@ __global__ void __launch_bounds__(320, 1)
   const WaitCtl ctl{abort_flag, p.timeout_ns};
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-#if FA_BWD_KEY_TILE_MAJOR
   // heaviest key tiles (the first ones under a causal mask) first, every (b, KV head) of a
   // key tile before the next key tile
   const int j = static_cast<int>(blockIdx.x) / (p.B * p.Hkv);
   const int bg = static_cast<int>(blockIdx.x) % (p.B * p.Hkv);
-#else
-  // the key tiles of one (b, KV head) next to each other: they share its Q / dO in L2
-  const int j = static_cast<int>(blockIdx.x) % p.n_tiles;
-  const int bg = static_cast<int>(blockIdx.x) / p.n_tiles;
-#endif
   const int g = bg % p.Hkv, b = bg / p.Hkv;
   const int k0 = 128 * j;
   // query tiles whose rows see some key of [k0, k0 + 127]

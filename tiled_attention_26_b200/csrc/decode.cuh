@@ -170,17 +170,9 @@ __device__ __forceinline__ void cp_async_wait_all() {
   asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
-#ifndef FA_DECODE_STAGES
-#define FA_DECODE_STAGES 2  // K/V stages of 128 keys in the shared-memory ring (3 CTAs per SM)
-#endif
-
-#ifndef FA_DECODE_MIN_CHUNK
-#define FA_DECODE_MIN_CHUNK 128  // keys; a multiple of 128
-#endif
-
-#ifndef FA_DECODE_PDL
-#define FA_DECODE_PDL 1  // launch the merge kernel as a programmatic dependent of the split kernel
-#endif
+// Shape constants of the decode kernels.
+constexpr int kDecodeStages = 2;      // K/V stages of 128 keys in the shared-memory ring (3 CTAs per SM)
+constexpr int kDecodeMinChunk = 128;  // smallest split, in keys; a multiple of 128
 
 // Shared-memory plan of the split kernel.  A stage holds 128 keys: the K and V code tiles
 // ([128 rows][kRow bytes], swizzled like the TMA box so that the row-per-lane fragment reads
@@ -188,7 +180,7 @@ __device__ __forceinline__ void cp_async_wait_all() {
 template <int D, int kBits>
 struct DecodeCfg {
   static constexpr int kT = 128;                  // keys per stage
-  static constexpr int kStages = FA_DECODE_STAGES;
+  static constexpr int kStages = kDecodeStages;
   static constexpr int kRow = D * kBits / 8;      // bytes of one key row of codes
   static constexpr int kTile = kT * kRow;         // bytes of one K or V code tile
   static constexpr int kStageBytes = 2 * kTile;
@@ -284,8 +276,8 @@ __global__ void __launch_bounds__(160, kBits == 8 ? 3 : 1) fa_decode_split_kerne
     }
   }
   // splits are whole stages (every stage starts on a multiple of 128 keys) of at least
-  // FA_DECODE_MIN_CHUNK keys: a short sequence takes few splits rather than many tiny ones
-  const int chunk = max(FA_DECODE_MIN_CHUNK,
+  // kDecodeMinChunk keys: a short sequence takes few splits rather than many tiny ones
+  const int chunk = max(kDecodeMinChunk,
                         ((len + p.splits - 1) / p.splits + C::kT - 1) / C::kT * C::kT);
   const int t_begin = min(len, split * chunk);
   const int t_end = min(len, t_begin + chunk);

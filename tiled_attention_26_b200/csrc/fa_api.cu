@@ -330,7 +330,7 @@ int launch_split_and_combine(const fa::DecodeParams& p, int keys, int outer, voi
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = FA_DECODE_PDL;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (cudaLaunchKernelEx(&cfg, fa::fa_decode_combine_kernel<D>, cp) != cudaSuccess)
@@ -568,13 +568,16 @@ const char* fa_status_string(int status) {
 }
 
 int fa_device_status(void* stream) {
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_CUDA;
+  // One host thread at a time: the taken value passes through one device variable.
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  fa::status_take_kernel<<<1, 1, 0, s>>>();
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return FA_ERR_CUDA;
   unsigned int v = 0;
-  if (cudaMemcpyFromSymbol(&v, fa::g_fa_device_status, sizeof v) != cudaSuccess) return FA_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&v, fa::g_fa_status_taken, sizeof v) != cudaSuccess) return FA_ERR_CUDA;
   if (v == 0) return FA_OK;
-  const unsigned int zero = 0;
-  if (cudaMemcpyToSymbol(fa::g_fa_device_status, &zero, sizeof zero) != cudaSuccess)
-    return FA_ERR_CUDA;
   if (v & fa::kDevStatusTimeout) return FA_ERR_TIMEOUT;
   return (v & fa::kDevStatusBadIndex) ? FA_ERR_DEVICE_INDEX : FA_ERR_CUDA;
 }

@@ -33,10 +33,6 @@
 
 namespace fa {
 
-#ifndef FA_REGS_SOFTMAX
-#define FA_REGS_SOFTMAX 216
-#endif
-
 struct PrefillParams {
   int B, Hq, Hkv, Sq, Skv;
   int G;       // query heads per KV head
@@ -82,10 +78,7 @@ struct PrefillCfg {
   static constexpr int kHalves = D / 64;          // 128-byte swizzle atoms along D
   static constexpr int kAtomBytes = 128 * 128;    // 128 rows x 128 bytes
   static constexpr int kTileBytes = 128 * D * 2;  // one 128-row bf16 tile
-#ifndef FA_KV_STAGES_D128
-#define FA_KV_STAGES_D128 4
-#endif
-  static constexpr int kStages = (D == 128) ? FA_KV_STAGES_D128 : 8;
+  static constexpr int kStages = (D == 128) ? 4 : 8;
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
@@ -109,7 +102,7 @@ struct PrefillCfg {
   static constexpr int kMaskBytes = 8 * 2 * kMaskSlotBytes;   // 32 KB
   static constexpr int kSmemBytesMask = kMaskOff + kMaskBytes + 1024;
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kRegsSoftmax = FA_REGS_SOFTMAX;
+  static constexpr uint32_t kRegsSoftmax = 216;
   // the rest of the 384 x 168 launch registers go to the producer / MMA warpgroup
   static constexpr uint32_t kRegsOther = ((168 * 384 - 2 * 128 * kRegsSoftmax) / 128) / 8 * 8;
   static constexpr int kMinLaunchRegs =
@@ -127,24 +120,6 @@ __device__ __forceinline__ int vis_lo(const PrefillParams& p, int i) {
 }
 __device__ __forceinline__ int vis_hi(const PrefillParams& p, int i) {
   return p.causal ? min(i + (p.Skv - p.Sq), p.Skv - 1) : p.Skv - 1;
-}
-
-#ifndef FA_EXP2_EMU_OF8
-#define FA_EXP2_EMU_OF8 0  // of every 8 column pairs, this many use exp2_fma on unmasked tiles
-#endif
-constexpr int kEmuOf8 = FA_EXP2_EMU_OF8;
-#ifndef FA_PACK_INT
-#define FA_PACK_INT 0  // 1: bf16 rounding with an integer add and a byte permute instead of cvt
-#endif
-
-// Two non-negative fp32 values -> bf16x2 (lo in the low half).
-__device__ __forceinline__ uint32_t pack_p(float lo, float hi) {
-#if FA_PACK_INT
-  // round half up on the magnitude (the values are >= 0), keep the upper halves
-  return prmt(__float_as_uint(lo) + 0x8000u, __float_as_uint(hi) + 0x8000u, 0x7632u);
-#else
-  return pack_bf16x2(lo, hi);
-#endif
 }
 
 // Row maximum of the 128 raw scores (3-input max, 8 independent chains).
@@ -165,7 +140,6 @@ __device__ __forceinline__ float row_max128(const uint32_t (&sv)[4][32]) {
 
 // p = 2^(s * sl2 - m_use) for the 64 columns of one half, written to TMEM as 32 bf16 pairs;
 // returns the fp32 sum of the half through acc (two packed partial sums).
-template <bool kEmu>
 __device__ __forceinline__ void exp_half(const uint32_t (&sv)[4][32], int half, float sl2,
                                          float m_use, uint32_t taddr, uint64_t& acc0,
                                          uint64_t& acc1) {
@@ -177,16 +151,11 @@ __device__ __forceinline__ void exp_half(const uint32_t (&sv)[4][32], int half, 
     const uint64_t x = f2_fma(f2(__uint_as_float(sv[col / 32][col % 32]),
                                  __uint_as_float(sv[(col + 1) / 32][(col + 1) % 32])),
                               scale2, negm2);
-    float x0, x1, a, c;
+    float x0, x1;
     f2_split(x, x0, x1);
-    if (kEmu && (k % 8) < kEmuOf8) {
-      exp2_fma_x2(x0, x1, a, c);
-    } else {
-      a = ex2(x0);
-      c = ex2(x1);
-    }
+    const float a = ex2(x0), c = ex2(x1);
     if (k & 1) acc1 = f2_add(acc1, f2(a, c)); else acc0 = f2_add(acc0, f2(a, c));
-    pk[k] = pack_p(a, c);
+    pk[k] = pack_bf16x2(a, c);
   }
   tmem_st32(taddr + 32 * half, pk);
 }
@@ -622,17 +591,15 @@ __global__ void __launch_bounds__(384, 1)
       }
       const float m_use = (m == -INFINITY) ? 0.f : m;
       // p = 2^(s * scale * log2(e) - m) as bf16 pairs over the S columns, one half at a time;
-      // each half is released to the MMA warp as soon as it is in TMEM.  Unmasked tiles take
-      // kEmuOf8 of every 8 pairs through exp2_fma (FMA pipe) to offload the MUFU pipe; masked
-      // tiles use MUFU only, so masked scores give exactly 0.
+      // each half is released to the MMA warp as soon as it is in TMEM.
       uint64_t acc0 = f2(0.f, 0.f), acc1 = f2(0.f, 0.f);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        if (need_mask || kMask) {
-          exp_half<false>(sv, half, sl2, m_use, trow + colS, acc0, acc1);
-        } else {
-          exp_half<true>(sv, half, sl2, m_use, trow + colS, acc0, acc1);
-        }
+        // (the two identical calls keep the register allocation of the plain path spill-free)
+        if (need_mask || kMask)
+          exp_half(sv, half, sl2, m_use, trow + colS, acc0, acc1);
+        else
+          exp_half(sv, half, sl2, m_use, trow + colS, acc0, acc1);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(C::kBarPFull + 2 * t + half));

@@ -17,6 +17,12 @@ namespace fa {
 // the definition lives here.
 enum : unsigned { kDevStatusTimeout = 1u, kDevStatusBadIndex = 2u };
 __device__ unsigned int g_fa_device_status = 0;
+// Where status_take_kernel leaves the word it took, for the host to read after a sync.
+__device__ unsigned int g_fa_status_taken = 0;
+
+// Reads and clears the status word in one atomic step (a report set between a separate read
+// and clear would be lost).
+__global__ void status_take_kernel() { g_fa_status_taken = atomicExch(&g_fa_device_status, 0u); }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -278,19 +284,6 @@ __device__ __forceinline__ void setmaxnreg_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-// 2^x on the FMA pipe, for x in [-125, 64] (callers clamp).  Range reduction x = n + f with
-// n = round(x) through the 1.5 * 2^23 rounding constant, f in [-1/2, 1/2]; 2^f from a degree-3
-// minimax polynomial (max relative error 7.5e-5, coefficients from exp2_poly.py); 2^n added to
-// the exponent field as an integer.
-__device__ __forceinline__ float exp2_fma(float x) {
-  const float t = x + 12582912.0f;
-  const float f = x - (t - 12582912.0f);
-  float p = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
-  p = fmaf(p, f, 0.6932609677314758f);
-  p = fmaf(p, f, 0.9999280571937561f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -321,25 +314,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
-}
-
-// exp2_fma on a packed pair (same range reduction and polynomial, f32x2 arithmetic).
-__device__ __forceinline__ void exp2_fma_x2(float x0, float x1, float& y0, float& y1) {
-  const uint64_t kMagic = f2(12582912.0f, 12582912.0f);
-  const uint64_t kNegMagic = f2(-12582912.0f, -12582912.0f);
-  const uint64_t kMinus1 = f2(-1.0f, -1.0f);
-  const uint64_t x = f2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-  const uint64_t t = f2_add(x, kMagic);
-  const uint64_t f = f2_fma(f2_add(t, kNegMagic), kMinus1, x);
-  uint64_t p = f2_fma(f2(0.0551716685295105f, 0.0551716685295105f), f,
-                      f2(0.2426111251115799f, 0.2426111251115799f));
-  p = f2_fma(p, f, f2(0.6932609677314758f, 0.6932609677314758f));
-  p = f2_fma(p, f, f2(0.9999280571937561f, 0.9999280571937561f));
-  float p0, p1, t0, t1;
-  f2_split(p, p0, p1);
-  f2_split(t, t0, t1);
-  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
