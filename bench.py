@@ -412,8 +412,9 @@ def cpu_baseline_decode(dev_inputs, w, budget_s: float, seed: int):
     import numpy as np
 
     import oracle
-    q, kq, vq, ks, vs = (t.cpu().numpy() for t in dev_inputs)
-    q = q.view(np.uint16) if q.dtype != np.uint16 else q
+    import torch
+    q = dev_inputs[0].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    kq, vq, ks, vs = (t.cpu().numpy() for t in dev_inputs[1:])
     G = w.Hq // w.Hkv
 
     def rows(n, s):
@@ -593,6 +594,29 @@ def run_only_prefill(args):
     return 0
 
 
+def run_only_masked(args):
+    """fa_fwd with the per-head additive bias mask on the MHA causal workload alone, one JSON
+    line (used to profile the masked prefill kernel)."""
+    import torch
+
+    import synthetic
+    import tiled_attention_26_b200 as fa
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    mv = measure_mask_variants(fa, synthetic, torch, dev, stream, steps=args.steps,
+                               warmup=args.warmup)
+    ms, flops = mv["masked"]
+    peaks, _ = load_peaks()
+    print(json.dumps({"metric": "masked attention forward TFLOP/s (4*D flops per visible pair)",
+                      "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_call": ms,
+                      "steps": args.steps, "warmup": args.warmup,
+                      "frac_of_burst": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+                      "config": {"workload": "mha_causal + per-head fp32 bias [1, 32, 4096, 4096]"}}),
+          flush=True)
+    return 0
+
+
 def run_only_backward(args):
     """fa_bwd on the MHA causal workload alone, one JSON line (used to profile the backward
     kernels without the other workloads resident on the device)."""
@@ -702,7 +726,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["backward", "prefill", "paged", "decode", "int4"],
+    ap.add_argument("--only", choices=["backward", "prefill", "paged", "decode", "int4", "masked"],
                     default=None,
                     help="time one further row on its own (for profiling); prints its own line")
     args = ap.parse_args()
@@ -718,6 +742,8 @@ def main():
         return run_only_decode(args)
     if args.only == "int4":
         return run_only_int4(args)
+    if args.only == "masked":
+        return run_only_masked(args)
 
     import torch
 

@@ -407,6 +407,13 @@ __global__ void __launch_bounds__(160, kBits == 8 ? 3 : 1) fa_decode_split_kerne
 
   // ============================ consumer warps 0..3 ============================
   const int g = lane >> 2, c = lane & 3;
+  // Key of slot k (0..15) of a 16-key group, the same for the K rows (QK m-rows), their scales
+  // and masks, and the V rows (PV k-index), so the product is unchanged.  4-bit code rows are 64
+  // bytes: with the identity, the PV fragment reads of keys 2c (c = 0..3) would all fall in the
+  // same half of their 128-byte lines (a 2-way bank conflict); flipping bit 0 when bit 1 is set
+  // spreads them over both halves and both swizzle groups while keeping each QK pair (2i, 2i+1)
+  // in different halves.
+  auto kslot = [](int k) { return kBits == 4 ? (k ^ ((k >> 1) & 1)) : k; };
 
   // ---- Q as the B operand of the QK mma, fp16, scaled by 2^eq per head (exact) ----
   // Thread c holds dims [QD*c, QD*c + QD) of its head, in the order its K fragment takes them
@@ -470,7 +477,7 @@ __global__ void __launch_bounds__(160, kBits == 8 ? 3 : 1) fa_decode_split_kerne
         uint32_t kw[2][QW];  // this thread's words of rows g and g + 8 of the group
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
-          const uint32_t row0 = (r_w + 16 * u + g + 8 * rr) * C::kRow + QD * kBits / 8 * c;
+          const uint32_t row0 = (r_w + 16 * u + kslot(g + 8 * rr)) * C::kRow + QD * kBits / 8 * c;
 #pragma unroll
           for (int w4 = 0; w4 < QW; w4 += 4) {
             if constexpr (QW >= 4) {
@@ -502,8 +509,8 @@ __global__ void __launch_bounds__(160, kBits == 8 ? 3 : 1) fa_decode_split_kerne
                           nib_hi16_f16x2(w1), qf[st][0], qf[st][1]);
           }
         }
-        const int rA = r_w + 16 * u + g, rB = rA + 8;
-        const int tA = T + 16 * u + g, tB = tA + 8;
+        const int rA = r_w + 16 * u + kslot(g), rB = r_w + 16 * u + kslot(g + 8);
+        const int tA = T + 16 * u + kslot(g), tB = T + 16 * u + kslot(g + 8);
         const float kA = lds32f(ks_s + 4 * rA), kB = lds32f(ks_s + 4 * rB);
         x[u][0] = tA < t_end ? sacc[0] * kA * sc0 : -INFINITY;
         x[u][1] = tA < t_end ? sacc[1] * kA * sc1 : -INFINITY;
@@ -549,8 +556,8 @@ __global__ void __launch_bounds__(160, kBits == 8 ? 3 : 1) fa_decode_split_kerne
       for (int u = 0; u < 2; ++u)
 #pragma unroll
         for (int rr = 0; rr < 2; ++rr) {
-          const int row = r_w + 16 * u + g + 8 * rr;
-          vsc[u][rr] = (T + 16 * u + g + 8 * rr < t_end) ? lds32f(vs_s + 4 * row) : 0.f;
+          const int row = r_w + 16 * u + kslot(g + 8 * rr);
+          vsc[u][rr] = (T + 16 * u + kslot(g + 8 * rr) < t_end) ? lds32f(vs_s + 4 * row) : 0.f;
           vmax = fmaxf(vmax, vsc[u][rr]);
         }
 #pragma unroll
@@ -589,7 +596,7 @@ __global__ void __launch_bounds__(160, kBits == 8 ? 3 : 1) fa_decode_split_kerne
         uint32_t r[4][VW];  // this thread's words of keys 2c, 2c+1, 2c+8, 2c+9 of the group
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
-          const int row = r_w + 16 * u + 2 * c + (q4 & 1) + 8 * (q4 >> 1);
+          const int row = r_w + 16 * u + kslot(2 * c + (q4 & 1) + 8 * (q4 >> 1));
           const uint32_t off = swz<C::kRow>(row * C::kRow + VB * g);
           if constexpr (VB == 16) {
             const uint4 x = lds128(vt + off);
