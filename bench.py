@@ -565,8 +565,8 @@ def weak_scaling_throughput(world: int, steps: int, work_per_step: float, max_ms
 
 
 def run_only_prefill(args):
-    """fa_fwd on the MHA causal workload alone, one JSON line (used to profile the prefill
-    kernel without the other workloads resident on the device)."""
+    """fa_fwd on one prefill workload alone (--workload, default the MHA causal one), one JSON
+    line (used to profile the prefill kernel without the other workloads resident)."""
     import torch
 
     import synthetic
@@ -574,12 +574,12 @@ def run_only_prefill(args):
     dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
-    w = synthetic.WORKLOADS["mha_causal"]
+    w = synthetic.WORKLOADS[args.workload]
     q, k, v = synthetic.make_qkv_torch(w, dev)
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.Sq), dtype=torch.float32, device=dev)
-    ms = time_calls(torch, stream, lambda: fa.fa_fwd(q, k, v, causal=True, scale=w.scale, o=o,
-                                                      lse=lse, stream=stream),
+    ms = time_calls(torch, stream, lambda: fa.fa_fwd(q, k, v, causal=w.causal, window=w.window,
+                                                      scale=w.scale, o=o, lse=lse, stream=stream),
                     args.steps, args.warmup)
     if fa.fa_device_status() != 0:
         raise RuntimeError("the prefill kernel reported a device-side error")
@@ -589,8 +589,7 @@ def run_only_prefill(args):
                       "value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                       "ms_per_call": ms, "steps": args.steps, "warmup": args.warmup,
                       "frac_of_burst": flops / (ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
-                      "config": {"workload": "mha_causal (B=2, H=32, S=4096, D=128, causal)"}}),
-          flush=True)
+                      "config": {"workload": args.workload}}), flush=True)
     return 0
 
 
@@ -723,6 +722,9 @@ def main():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mha_causal",
+                    choices=["mha_causal", "gqa_causal", "gqa_sw512", "mqa_causal"],
+                    help="prefill workload of --only prefill")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-budget", type=float, default=12.0, help="seconds of oracle work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
