@@ -48,8 +48,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from ncu, keyed by the sha256 of the
 # kernel sources they were taken on; a kernel edited since then reports traffic = null.
 NCU_TRAFFIC = {
-    # profiles/fa_prefill_kernel_mha_causal.md: 535,730,176 B read + 48,052,736 B written
-    "prefill": {"bb30a856dfed342d": 583_782_912},
+    # profiles/fa_prefill_kernel_mha_causal.md: 534,377,472 B read + 48,006,144 B written
+    "prefill": {"753bf7e28f87f0e5": 582_383_616},
     # profiles/fa_decode_split_kernel_decode_int8.md: 1,107,942,400 B read + 10,583,808 B written
     "decode": {"a06a790a147221ec": 1_118_526_208},
     # profiles/fa_decode_split_kernel_decode_int8_paged.md: 424,260,352 B read + 4,880,128 B

@@ -55,6 +55,14 @@ def test_decode_8bit_kernels_fit_three_ctas_per_sm(kernels):
             assert v["spill"] <= 32, (name, v)
 
 
+def test_decode_4bit_kernels_fit_three_ctas_per_sm(kernels):
+    # the 4-bit kernels run the same 160-thread, 3-CTA-per-SM configuration
+    for name, v in _select(kernels, "_ZN2fa22fa_decode_split_kernelI").items():
+        if "ELi4EE" in name:
+            assert v["regs"] * 160 * 3 <= REGFILE, (name, v)
+            assert v["spill"] <= 32, (name, v)
+
+
 def test_prefill_launch_registers_match_the_warpgroup_split(kernels):
     # 384 threads at 168 registers: softmax warpgroups 2 x 128 x 216 plus the producer / MMA
     # warpgroup 128 x 72 use exactly the launch's 384 x 168
