@@ -50,11 +50,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NCU_TRAFFIC = {
     # profiles/fa_prefill_kernel_mha_causal.md: 534,377,472 B read + 48,006,144 B written
     "prefill": {"753bf7e28f87f0e5": 582_383_616},
-    # profiles/fa_decode_split_kernel_decode_int8.md: 1,107,942,400 B read + 10,583,808 B written
-    "decode": {"a06a790a147221ec": 1_118_526_208},
-    # profiles/fa_decode_split_kernel_decode_int8_paged.md: 424,260,352 B read + 4,880,128 B
+    # profiles/fa_decode_split_kernel_decode_int8.md: 1,108,583,680 B read + 14,467,328 B written
+    "decode": {"db2267d0a6c42aac": 1_123_051_008},
+    # profiles/fa_decode_split_kernel_decode_int8_paged.md: 424,287,744 B read + 4,637,696 B
     # written
-    "paged_decode": {"a06a790a147221ec": 429_140_480},
+    "paged_decode": {"db2267d0a6c42aac": 428_925_440},
 }
 
 

@@ -620,6 +620,9 @@ __global__ void __launch_bounds__(384, 1)
       bool ok = mbar_wait(bar(C::kBarOFinal + t), 0, ctl);
       have_o = __all_sync(0xffffffffu, ok);
       tc_fence_after();
+    } else {
+      // no product ran for this tile: the Q copy into its staging buffer may still be landing
+      mbar_wait(bar(C::kBarQ), 0, ctl);
     }
     const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
     const uint32_t stage = sQ + t * C::kTileBytes;  // Q tile t is no longer read
