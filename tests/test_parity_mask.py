@@ -112,6 +112,31 @@ def test_global_local_full_oracle(fa, case):
     check_lse(lse.cpu().numpy().astype(np.float64), l_ref, what)
 
 
+MASKED_GLOBAL = [
+    # B, Hq, Hkv, S, D, global tokens, W, mask kind: the mask tensor and global + local
+    # attention together (the key tiles between the global ones and the band are skipped, so the
+    # mask staging follows the same gaps)
+    (1, 4, 2, 700, 128, 150, 64, "bias1h"),
+    (2, 2, 1, 1000, 64, 3, 32, "holes"),
+]
+
+
+@pytest.mark.parametrize("case", MASKED_GLOBAL)
+def test_masked_global_local_full_oracle(fa, case):
+    import torch
+    B, Hq, Hkv, S, D, G, W, kind = case
+    q, k, v = _qkv(B, Hq, Hkv, S, S, D, 850 + S)
+    mask = _mask(kind, B, Hq, S, S, 11)
+    s = float(np.float32(1 / math.sqrt(D)))
+    o, lse = fa.fa_fwd(to_dev_bf16(q), to_dev_bf16(k), to_dev_bf16(v), causal=True, window=W,
+                       scale=s, n_global=G, mask=torch.from_numpy(mask).cuda())
+    assert fa.fa_device_status() == 0
+    o_ref, l_ref = oracle.attn_ext(q, k, v, s, 1, W, G, mask)
+    what = f"mask {kind} + global G{G} W{W} B{B} Hq{Hq} Hkv{Hkv} S{S} D{D}"
+    check_o(o_to_f64(o), o_ref, what)
+    check_lse(lse.cpu().numpy().astype(np.float64), l_ref, what)
+
+
 def test_global_local_full_size_sampled(fa):
     # the GQA sliding-window workload (B=3, Hq=32, Hkv=8, S=4096, W=512) with 64 global tokens
     import torch
