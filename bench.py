@@ -979,7 +979,8 @@ def main():
                 "frac": mv["global_local"][1] / (mv["global_local"][0] * 1e-3) / 1e12 / tpeak},
             "backward": {
                 "workload": "mha_causal (B=2, H=32, S=4096, D=128, causal): fa_bwd after fa_fwd",
-                "kernels": "fa_bwd_prep_kernel + fa_bwd_dkdv_kernel<128> + fa_bwd_dq_kernel<128>",
+                "kernels": "fa_bwd_prep_kernel + fa_bwd_kernel<128> (dK, dV and the dQ shares) + "
+                           "fa_bwd_dq_finalize_kernel",
                 "ms_per_call": bw_ms, "flops_per_call": bw_flops,
                 "achieved": bw_flops / (bw_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "frac": bw_flops / (bw_ms * 1e-3) / 1e12 / tpeak},

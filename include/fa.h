@@ -122,10 +122,16 @@ FA_API int fa_fwd_ext(const void* q, const void* k, const void* v, void* o, floa
  *   dq          bf16 [B, Sq, Hq, D]  written
  *   dk, dv      bf16 [B, Skv, Hkv, D] written; for GQA / MQA they sum over the query heads that
  *               read each KV head
- *   workspace   at least fa_bwd_workspace_bytes(B, Hq, Sq) bytes (per-row D = dO . O and the
- *               log-sum-exp in log2 units); contents on entry do not matter.
- * Other arguments as for fa_fwd.  Three kernels run in order on `stream`; none uses atomics, so
- * the result is deterministic.  Returns FA_OK or an fa_status error code.
+ *   workspace   at least fa_bwd_workspace_bytes(B, Hq, Sq) bytes, 16-byte aligned: per-row
+ *               D = dO . O and the log-sum-exp in log2 units, then an fp32 dQ accumulator
+ *               [B, Sq, Hq, 128] (sized for D = 128 whatever D is); contents on entry do not
+ *               matter.
+ * Other arguments as for fa_fwd.  Three kernels run in order on `stream`: a per-row pass (D, L,
+ * and the accumulator zeroed), one kernel per (b, KV head, 128-key tile) that writes dK and dV
+ * and adds the tile's share of dQ into the accumulator (TMA tensor reductions), and a pass that
+ * scales the accumulator and rounds it to bf16.  dK and dV are deterministic; dQ is a sum of
+ * fp32 shares whose order depends on timing, so it can differ between runs in its last bits.
+ * Returns FA_OK or an fa_status error code.
  */
 FA_API size_t fa_bwd_workspace_bytes(int B, int Hq, int Sq);
 FA_API int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,

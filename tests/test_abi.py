@@ -118,7 +118,8 @@ def test_bwd_rejects(L, kw, code):
 
 
 def test_bwd_workspace_bytes(L):
-    assert fa.fa_bwd_workspace_bytes(2, 4, 300) == 2 * 2 * 4 * 384 * 4
+    # -L log2(e) and -D per padded row, then the fp32 dQ accumulator [B, Sq, Hq, 128]
+    assert fa.fa_bwd_workspace_bytes(2, 4, 300) == 2 * 2 * 4 * 384 * 4 + 2 * 300 * 4 * 128 * 4
     assert fa.fa_bwd_workspace_bytes(0, 4, 300) == 0
 
 

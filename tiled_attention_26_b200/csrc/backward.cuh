@@ -5,16 +5,19 @@
 // recomputation section).  With L the row log-sum-exp and D_i = dO_i . O_i:
 //   P_ij = exp(scale q_i.k_j - L_i),  dP_ij = dO_i . v_j,  dS_ij = P_ij (dP_ij - D_i)
 //   dV_j = sum_i P_ij dO_i,  dK_j = scale sum_i dS_ij q_i,  dQ_i = scale sum_j dS_ij k_j
-// Three kernels, none with atomics:
+// Three kernels:
 //   fa_bwd_prep_kernel   -D_i and -L_i * log2(e) per (b, h, i) into a padded workspace
-//                        (padding rows get L = +inf, D = 0: they contribute nothing);
-//   fa_bwd_dkdv_kernel   one CTA per (b, KV head, 128-key tile): S^T = K Q^T and
-//                        dP^T = V dO^T per (query head of the group, 128-query tile), then
-//                        dV += P^T dO and dK += dS^T Q with P and dS in TMEM (GQA heads summed
-//                        in TMEM), one bf16 store of dK and dV at the end;
-//   fa_bwd_dq_kernel     one CTA per 128-row Q tile (query heads packed into rows as in the
-//                        forward pass): S = Q K^T and dP = dO V^T per key tile, then
-//                        dQ += dS K with dS in TMEM.
+//                        (padding rows get L = +inf, D = 0: they contribute nothing), and the
+//                        row's fp32 dQ accumulator set to zero;
+//   fa_bwd_kernel        one CTA per (b, KV head, 128-key tile): per (query head of the group,
+//                        128-query tile) S^T = K Q^T and dP^T = V dO^T, then dV += P^T dO,
+//                        dK += dS^T Q (GQA heads summed in TMEM, one bf16 store of dK and dV at
+//                        the end) and the tile's share of dQ, dS K, staged in the unit's own
+//                        (no longer read) Q and dO buffers and added into the fp32 accumulator
+//                        by TMA tensor reductions (so S and dP are computed once per (query,
+//                        key) tile);
+//   fa_bwd_dq_finalize_kernel  dQ = scale * accumulator, rounded to bf16.
+// dK and dV are deterministic; dQ sums the key tiles' shares in the order the reductions land.
 // Warp roles (320 threads): warps 0-7 elementwise (thread = row = TMEM lane of its quadrant;
 // warps w and w + 4 share a quadrant and take one half of the columns each), warp 8 TMA
 // producer, warp 9 TMEM allocation + tcgen05.mma issue from one thread.
@@ -29,7 +32,7 @@ struct BwdParams {
   int B, Hq, Hkv, Sq, Skv;
   int G, Gp, NP;
   int Sq_pad;          // rows of the per-(b, h) workspace vectors (multiple of 128)
-  int n_tiles;         // dQ: 128-row Q tiles per (b, KV head, head pack); dK/dV: key tiles
+  int n_tiles;         // key tiles
   float scale;         // softmax scale
   float scale_log2;    // scale * log2(e)
   int causal, window;
@@ -38,6 +41,8 @@ struct BwdParams {
   const float* lse;      // natural log [B, Hq, Sq]
   float* lse2;           // workspace [B * Hq, Sq_pad]: -L * log2(e)
   float* delta;          // workspace [B * Hq, Sq_pad]: -D
+  float* dq_acc;         // workspace [B, Sq, Hq, D] fp32: sum over key tiles of dS K
+  uint16_t* dq;          // bf16 [B, Sq, Hq, D] output
   uint64_t timeout_ns;
 };
 
@@ -48,35 +53,35 @@ struct BwdCfg {
   static constexpr int kAtomBytes = 128 * 128;
   static constexpr int kTileBytes = 128 * D * 2;
   static constexpr uint32_t kTmemCols = 512;
-  // dQ kernel: Q and dO tiles, then a K/V ring
-  static constexpr int kQStages = (D == 128) ? 4 : 8;
-  static constexpr int kQOff = 0;
-  static constexpr int kDOOff = kTileBytes;
-  static constexpr int kQKVOff = 2 * kTileBytes;
-  static constexpr int kQBarOff = kQKVOff + kQStages * kTileBytes;
-  // barriers: in_full, kv_full[S], kv_empty[S], sdp_full, sdp_free, ds_ready, dq_done,
-  // o_final, drain
-  static constexpr int kQNumBars = 7 + 2 * kQStages;
-  static constexpr int kQMiscOff = kQBarOff + 8 * kQNumBars;
-  static constexpr int kQSmemBytes = kQMiscOff + 16 + 1024;
-  // dK/dV kernel: K and V tiles, then a ring of (Q, dO, L, D) units
+  // K and V tiles, then a ring of (Q, dO, L, D) units
   static constexpr int kUStages = (D == 128) ? 2 : 4;
   static constexpr int kUnitBytes = 2 * kTileBytes + 2 * 128 * 4;
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kTileBytes;
   static constexpr int kUOff = 2 * kTileBytes;
-  static constexpr int kUBarOff = kUOff + kUStages * kUnitBytes;
-  // barriers: kv_full, u_full[S] (Q and the vectors), u_empty[S], s_full, dp_full, p_ready,
-  // ds_ready, o_final, drain, u_do[S] (dO)
-  static constexpr int kUNumBars = 7 + 3 * kUStages;
+  // dS^T (bf16, 128 keys x 128 queries as two 128-byte swizzle atoms of 64 queries) is the A
+  // operand of dK += dS^T Q (K-major) and of dQ = dS K (read MN-major); it has a buffer of its
+  // own.  A unit's dQ share (128 query rows x D fp32) is then staged for the TMA reductions in
+  // two halves: dims [0, D/2) over the unit's dO tile, dims [D/2, D) over the dS^T buffer (both
+  // free once dK, the last product reading them, has run).
+  static constexpr int kDSOff = kUOff + kUStages * kUnitBytes;
+  static constexpr int kStgBytes = 128 * (D / 2) * 4;
+  static_assert(kStgBytes <= 2 * kAtomBytes, "dQ staging half over the dS^T buffer");
+  static constexpr int kUBarOff = kDSOff + 2 * kAtomBytes;
+  // barriers: kv_full, u_full[S] (Q and the vectors), q_empty[S], s_full, dp_full, p_ready,
+  // ds_ready, o_final, drain, u_do[S] (dO), dq_full, dq_free, dk_done, do_empty[S], x_free
+  static constexpr int kUNumBars = 11 + 4 * kUStages;
   static constexpr int kUMiscOff = kUBarOff + 8 * kUNumBars;
-  static constexpr int kUSmemBytes = kUMiscOff + 16 + 1024;
+  // (no slack for aligning the base: the kernel requires the dynamic shared memory to start
+  // 1024-byte aligned, checks it and reports a device error otherwise)
+  static constexpr int kUSmemBytes = kUMiscOff + 16;
+  static_assert(kUSmemBytes <= 227 * 1024, "backward kernel over the shared memory");
 };
 
 // ---------------------------------------------------------------------------------------
 // -D_i = -dO_i . O_i and -L_i * log2(e) per (b, h, i) row, D / 8 lanes per row (stored negated
 // so the kernels add them); padding rows past Sq get L = +inf and D = 0.  Rows with L = -inf (no
-// visible key) also get +inf: their P is 0.
+// visible key) also get +inf: their P is 0.  The row's dQ accumulator is zeroed.
 // ---------------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdParams p) {
@@ -116,6 +121,13 @@ __global__ void __launch_bounds__(256) fa_bwd_prep_kernel(const BwdParams p) {
     p.lse2[row] = -l2;
     p.delta[row] = (i < p.Sq) ? -acc : 0.f;
   }
+  // this row's fp32 dQ accumulator starts at zero (8 floats per lane)
+  if (valid && i < p.Sq) {
+    float4* z = reinterpret_cast<float4*>(
+        p.dq_acc + ((static_cast<size_t>(b) * p.Sq + i) * p.Hq + h) * D + 8 * sub);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 }
 
 // Query token i sees key k (bottom-right causal alignment, window of W keys).
@@ -128,27 +140,35 @@ __device__ __forceinline__ bool bwd_visible(const BwdParams& p, int i, int k) {
 }
 
 // ---------------------------------------------------------------------------------------
-// dK, dV: one CTA per (b, KV head g, key tile j).
+// One CTA per (b, KV head g, key tile j): dK and dV of the tile, and its share of dQ.
 // ---------------------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(320, 1)
-    fa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
-                       const __grid_constant__ CUtensorMap tm_k,
-                       const __grid_constant__ CUtensorMap tm_v,
-                       const __grid_constant__ CUtensorMap tm_do,
-                       const __grid_constant__ CUtensorMap tm_vec,
-                       const __grid_constant__ CUtensorMap tm_dk,
-                       const __grid_constant__ CUtensorMap tm_dv, const BwdParams p) {
+    fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                  const __grid_constant__ CUtensorMap tm_v,
+                  const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_vec,
+                  const __grid_constant__ CUtensorMap tm_dk,
+                  const __grid_constant__ CUtensorMap tm_dv,
+                  const __grid_constant__ CUtensorMap tm_dqacc, const BwdParams p) {
   using C = BwdCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // 128-byte swizzled TMA boxes need 1024-byte aligned shared memory, and this kernel has no
+  // room to align the base itself
+  if ((smem_u32(smem_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicOr(&g_fa_device_status, kDevStatusLayout);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   const uint32_t sb = smem_u32(smem);
   auto bar = [&](int idx) { return sb + C::kUBarOff + 8u * idx; };
   constexpr int kBarKV = 0, kBarUFull = 1, kBarUEmpty = 1 + C::kUStages;
   constexpr int kBarS = 1 + 2 * C::kUStages, kBarDP = kBarS + 1, kBarP = kBarS + 2,
                 kBarDS = kBarS + 3, kBarO = kBarS + 4, kBarDrain = kBarS + 5,
-                kBarUDo = kBarS + 6;
+                kBarUDo = kBarS + 6, kBarDQFull = kBarUDo + C::kUStages,
+                kBarDQFree = kBarDQFull + 1, kBarDKDone = kBarDQFull + 2,
+                kBarDOEmpty = kBarDQFull + 3, kBarXFree = kBarDOEmpty + C::kUStages;
+  static_assert(kBarXFree + 1 == C::kUNumBars, "barrier count");
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kUMiscOff);
   int* abort_flag = reinterpret_cast<int*>(smem + C::kUMiscOff + 4);
   const WaitCtl ctl{abort_flag, p.timeout_ns};
@@ -171,7 +191,10 @@ __global__ void __launch_bounds__(320, 1)
 
   if (threadIdx.x == 0) {
     for (int x = 0; x < C::kUNumBars; ++x)
-      mbar_init(bar(x), (x == kBarP || x == kBarDS) ? 256 : 1);
+      mbar_init(bar(x), (x == kBarP || x == kBarDS || x == kBarDQFree) ? 256
+                        : ((x >= kBarDOEmpty && x < kBarDOEmpty + C::kUStages) || x == kBarXFree)
+                            ? 8
+                            : 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -183,7 +206,8 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  constexpr uint32_t colS = 0, colDP = 128, colDV = 256, colDK = 256 + D;
+  // dQ of a unit accumulates over dP^T's columns once the elementwise warps have read dP^T
+  constexpr uint32_t colS = 0, colDP = 128, colDQ = 128, colDV = 256, colDK = 256 + D;
 
   if (warp == 8) {
     // ============ producer ============
@@ -198,6 +222,8 @@ __global__ void __launch_bounds__(320, 1)
       int issued = 0;
       for (int u = 0; u < n_units; ++u) {
         const int s = u % C::kUStages;
+        // Q and the vectors are free once dK of the stage's previous unit has run; dO (which
+        // also held that unit's dS^T and half its dQ staging) once the reductions have read it
         if (u >= C::kUStages &&
             !mbar_wait(bar(kBarUEmpty + s), ((u / C::kUStages) - 1) & 1, ctl))
           break;
@@ -213,12 +239,17 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t vb = base + 2 * C::kTileBytes;
         tma_load_3d(vb, &tm_vec, bar(kBarUFull + s), i0, b * p.Hq + h, 0);
         tma_load_3d(vb + 512, &tm_vec, bar(kBarUFull + s), i0, b * p.Hq + h, 1);
+        // (copies in flight from here on are waited for below, even if dO is never started:
+        // that wait then runs out)
+        issued = u + 1;
+        if (u >= C::kUStages &&
+            !mbar_wait(bar(kBarDOEmpty + s), ((u / C::kUStages) - 1) & 1, ctl))
+          break;
         mbar_arrive_expect_tx(bar(kBarUDo + s), C::kTileBytes);
 #pragma unroll
         for (int hf = 0; hf < C::kHalves; ++hf)
           tma_load_4d(base + C::kTileBytes + hf * C::kAtomBytes, &tm_do, bar(kBarUDo + s),
                       64 * hf, h, i0, b);
-        issued = u + 1;
       }
       volatile int zero = 0;
       const WaitCtl drain_ctl{&zero, p.timeout_ns};
@@ -233,7 +264,10 @@ __global__ void __launch_bounds__(320, 1)
     // ============ MMA issuer ============
     if (lane == 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
+      // A K-major (or in TMEM), B MN-major
       constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);
+      // A and B both MN-major (bit 15: A major)
+      constexpr uint32_t idesc_dq = idesc_bf16_f32(128, D, true) | (1u << 15);
       // D[tmem] = A_tile (K-major rows) . B_tile^T, K = D
       auto mma_rows = [&](uint32_t d, uint32_t a, uint32_t bt) {
 #pragma unroll
@@ -243,24 +277,44 @@ __global__ void __launch_bounds__(320, 1)
                   idesc_s, kk > 0 ? 1u : 0u);
         }
       };
-      // D[tmem] (+)= A[tmem bf16, 128 x 128] . B_tile (MN-major, K = the tile's 128 rows);
-      // A's queries 0-63 sit in columns [a_col, a_col + 32), queries 64-127 in
-      // [a_col + 64, a_col + 96)
-      auto mma_acc = [&](uint32_t d, uint32_t a_col, uint32_t bt, bool first) {
+      // dV += P^T dO: A = P^T in TMEM (queries 0-63 in columns [colS, colS + 32), queries
+      // 64-127 in [colS + 64, colS + 96)), B = the dO tile (MN-major, K = its 128 rows)
+      auto mma_dv = [&](uint32_t dot, bool first) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tmem + d, tmem + a_col + 64 * (kk / 4) + 8 * (kk % 4),
-                  smem_desc_sw128(bt + kk * 16 * 128, C::kAtomBytes, 1024), idesc_acc,
+          umma_ts(tmem + colDV, tmem + colS + 64 * (kk / 4) + 8 * (kk % 4),
+                  smem_desc_sw128(dot + kk * 16 * 128, C::kAtomBytes, 1024), idesc_acc,
                   (first && kk == 0) ? 0u : 1u);
       };
-      // Order: S(0) dP(0) | dV(u) S(u+1) | dK(u) dP(u+1) | ...: the tensor core works on the
-      // next unit's products while the elementwise warps turn S into P and dP into dS.
+      // dK += dS^T Q: A = dS^T (K-major: key rows, 16 queries per step), B = the Q tile
+      // (MN-major, K = its 128 rows)
+      auto mma_dk = [&](uint32_t ds, uint32_t qt, bool first) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ss(tmem + colDK,
+                  smem_desc_sw128(ds + (kk / 4) * C::kAtomBytes + (kk % 4) * 32, 16, 1024),
+                  smem_desc_sw128(qt + kk * 16 * 128, C::kAtomBytes, 1024), idesc_acc,
+                  (first && kk == 0) ? 0u : 1u);
+      };
+      // dQ = dS K over this key tile: A = dS (MN-major: the dS^T tile read with the queries
+      // contiguous, 16 keys per step), B = the K tile (MN-major, K = its 128 key rows)
+      auto mma_dq = [&](uint32_t ds) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ss(tmem + colDQ, smem_desc_sw128(ds + kk * 16 * 128, C::kAtomBytes, 1024),
+                  smem_desc_sw128(sb + C::kKOff + kk * 16 * 128, C::kAtomBytes, 1024), idesc_dq,
+                  kk > 0 ? 1u : 0u);
+      };
+      // Order: S(0) dP(0) | dV(u) S(u+1) dQ(u) dK(u) dP(u+1) | ...: the tensor core works on the
+      // next unit's S while the elementwise warps turn dP into dS; dQ(u) goes first so that its
+      // read-out overlaps dK(u); dP(u+1) waits until dQ(u) (which shares its columns) has been
+      // read out.
       auto unit_tiles = [&](int u, uint32_t& qt, uint32_t& dot) {
         qt = sb + C::kUOff + (u % C::kUStages) * C::kUnitBytes;
         dot = qt + C::kTileBytes;
       };
       // (waits on copies into shared memory need no tcgen05 fence: the MMAs read through the
-      // async proxy that wrote them; waits on TMEM written by other warps do)
+      // async proxy that wrote them; waits on TMEM or shared memory written by other warps do)
       bool ok = n_units > 0 && mbar_wait(bar(kBarKV), 0, ctl);
       if (ok && (ok = mbar_wait(bar(kBarUFull), 0, ctl))) {
         uint32_t qt, dot;
@@ -278,7 +332,7 @@ __global__ void __launch_bounds__(320, 1)
         const bool nxt = u + 1 < n_units;
         if (!(ok = mbar_wait(bar(kBarP), u & 1, ctl))) break;
         tc_fence_after();
-        mma_acc(colDV, colS, dot, u == 0);    // dV += P^T dO
+        mma_dv(dot, u == 0);                  // dV += P^T dO
         if (nxt) {
           if (!(ok = mbar_wait(bar(kBarUFull + (u + 1) % C::kUStages), ((u + 1) / C::kUStages) & 1, ctl)))
             break;
@@ -288,12 +342,18 @@ __global__ void __launch_bounds__(320, 1)
         }
         if (!(ok = mbar_wait(bar(kBarDS), u & 1, ctl))) break;
         tc_fence_after();
-        mma_acc(colDK, colDP, qt, u == 0);    // dK += dS^T Q
-        tc_commit(bar(kBarUEmpty + u % C::kUStages));
+        const uint32_t ds = sb + C::kDSOff;
+        mma_dq(ds);                           // this tile's dQ share = dS K
+        tc_commit(bar(kBarDQFull));
+        mma_dk(ds, qt, u == 0);               // dK += dS^T Q
+        tc_commit(bar(kBarDKDone));
+        tc_commit(bar(kBarUEmpty + u % C::kUStages));  // Q (the elementwise warps free dO)
         if (nxt) {
+          if (!(ok = mbar_wait(bar(kBarDQFree), u & 1, ctl))) break;
+          tc_fence_after();
           if (!(ok = mbar_wait(bar(kBarUDo + (u + 1) % C::kUStages), ((u + 1) / C::kUStages) & 1, ctl)))
             break;
-          mma_rows(colDP, sb + C::kVOff, don);  // dP^T of the next unit (after dK read dS)
+          mma_rows(colDP, sb + C::kVOff, don);  // dP^T of the next unit (after dQ was read)
           tc_commit(bar(kBarDP));
         }
       }
@@ -304,14 +364,27 @@ __global__ void __launch_bounds__(320, 1)
       mbar_wait(bar(kBarDrain), 0, drain_ctl);
     }
   } else {
-    // ============ elementwise: thread = key row; this warp's half of the query columns ====
+    // ============ elementwise: thread = key row (S^T, dP^T) / query row (dQ); this warp's
+    // half of the columns ============
     const int wq = warp & 3, ch = warp >> 2;
     const int r = 32 * wq + lane;
     const int key = k0 + r;
     const uint32_t trow = tmem + (static_cast<uint32_t>(32 * wq) << 16);
     const uint64_t sl2 = f2(p.scale_log2, p.scale_log2);
+    // Lane 0: the stage whose dQ reductions were issued last and whose release to the producer
+    // waits until the reductions have read it (done after the next unit's P, so the reductions
+    // overlap that work), or -1.
+    int pend_s = -1;
+    auto release_pending = [&]() {
+      if (lane == 0 && pend_s >= 0) {
+        tma_store_wait_read_all();
+        mbar_arrive(bar(kBarDOEmpty + pend_s));
+      }
+      pend_s = -1;
+    };
     for (int u = 0; u < n_units; ++u) {
       const int s = u % C::kUStages;
+      const int h = g * p.G + u / n_qt;
       const int i0 = 128 * (qt_lo + u % n_qt);
       // -L log2(e) and -D of the unit's 128 queries (broadcast reads, four at a time)
       const float4* vl = reinterpret_cast<const float4*>(smem + C::kUOff + s * C::kUnitBytes +
@@ -353,16 +426,18 @@ __global__ void __launch_bounds__(320, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(kBarP));
-      // ---- dS = P (dP^T - D) ----
+      release_pending();
+      if (lane == 0) mbar_arrive(bar(kBarXFree));  // this warp's earlier reductions were read
+      // ---- dS = P (dP^T - D), bf16, into shared memory as row r (key) of the dS^T tile ----
       ok = mbar_wait(bar(kBarDP), u & 1, ctl);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
+      uint32_t ds[32];
       {
         uint32_t dv[64];
         tmem_ld32(trow + colDP + 64 * ch, *reinterpret_cast<uint32_t(*)[32]>(dv));
         tmem_ld32(trow + colDP + 64 * ch + 32, *reinterpret_cast<uint32_t(*)[32]>(dv + 32));
         tmem_wait_ld();
-        uint32_t ds[32];
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
           const float4 nd = vd[q];
@@ -378,12 +453,73 @@ __global__ void __launch_bounds__(320, 1)
           ds[2 * q] = pack_bf16x2(d0, d1);
           ds[2 * q + 1] = pack_bf16x2(d2, d3);
         }
-        tmem_st32(trow + colDP + 64 * ch, ds);
       }
-      tmem_wait_st();
+      // the dS^T buffer held the previous unit's dQ staging: every warp's reductions of it
+      // have been read (each warp's lane 0 waited in release_pending) before anyone writes
+      ok = mbar_wait(bar(kBarXFree), u & 1, ctl);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      {
+        // atom ch holds queries 64 ch .. 64 ch + 63; 16-byte chunk c of row r (queries
+        // 8c .. 8c + 7 of the atom) sits at chunk c ^ (r & 7), the 128-byte swizzle
+        uint8_t* row_ptr = smem + C::kDSOff + ch * C::kAtomBytes + r * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<uint4*>(row_ptr + 16 * (c ^ (r & 7))) =
+              make_uint4(ds[4 * c], ds[4 * c + 1], ds[4 * c + 2], ds[4 * c + 3]);
+      }
+      fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(kBarDS));
+      // ---- this unit's dQ share: TMEM lane = query row r, this warp's half of the dims ----
+      ok = mbar_wait(bar(kBarDQFull), u & 1, ctl);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      uint32_t qv[D / 2];
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c)
+        tmem_ld32(trow + colDQ + (D / 2) * ch + 32 * c,
+                  *reinterpret_cast<uint32_t(*)[32]>(qv + 32 * c));
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(bar(kBarDQFree));
+      // the staging below overwrites Q and dS^T, which dK += dS^T Q reads
+      ok = mbar_wait(bar(kBarDKDone), u & 1, ctl);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      {
+        // Stage this warp's 32 rows x D/2 dims: boxes of 32 rows x 32 fp32 (128 bytes a row,
+        // 128-byte swizzle), box (wq, k) at 4 KB * (k * 4 + wq) of the unit's dO tile (ch = 0)
+        // or of the dS^T buffer (ch = 1), which every product has finished reading (dK is the
+        // last); then one lane adds them into the accumulator (the dO tile goes back to the
+        // producer once they are read).
+        constexpr int kBoxes = D / 64;
+        const uint32_t st_base =
+            ch ? C::kDSOff : C::kUOff + s * C::kUnitBytes + C::kTileBytes;
+#pragma unroll
+        for (int k = 0; k < kBoxes; ++k) {
+          uint8_t* row_ptr = smem + st_base + 4096 * (k * 4 + wq) + lane * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(row_ptr + 16 * (c ^ (lane & 7))) =
+                make_uint4(qv[32 * k + 4 * c], qv[32 * k + 4 * c + 1], qv[32 * k + 4 * c + 2],
+                           qv[32 * k + 4 * c + 3]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int t0 = i0 + 32 * wq;  // first query row of this warp
+          if (t0 < p.Sq) {
+#pragma unroll
+            for (int k = 0; k < kBoxes; ++k)
+              tma_reduce_add_4d(&tm_dqacc, sb + st_base + 4096 * (k * 4 + wq),
+                                (D / 2) * ch + 32 * k, h, t0, b);
+            tma_store_commit();
+          }
+        }
+        pend_s = s;
+        __syncwarp();
+      }
     }
+    release_pending();
     // ---- epilogue: warps 0-3 write dV, warps 4-7 scale * dK: bf16 -> swizzled smem (the
     // V / K tiles) -> TMA ----
     bool have = false;
@@ -442,278 +578,20 @@ __global__ void __launch_bounds__(320, 1)
 }
 
 // ---------------------------------------------------------------------------------------
-// dQ: one CTA per 128-row Q tile; row r = (token t0 + r / Gp, head h0 + r % Gp).
+// dQ = scale * accumulator -> bf16, eight elements per thread.
 // ---------------------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(320, 1)
-    fa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q,
-                     const __grid_constant__ CUtensorMap tm_k,
-                     const __grid_constant__ CUtensorMap tm_v,
-                     const __grid_constant__ CUtensorMap tm_do,
-                     const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
-  using C = BwdCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  const uint32_t sb = smem_u32(smem);
-  auto bar = [&](int idx) { return sb + C::kQBarOff + 8u * idx; };
-  constexpr int kBarIn = 0, kBarKVFull = 1, kBarKVEmpty = 1 + C::kQStages;
-  constexpr int kBarSDP = 1 + 2 * C::kQStages, kBarFree = kBarSDP + 1, kBarDS = kBarSDP + 2,
-                kBarDQ = kBarSDP + 3, kBarO = kBarSDP + 4, kBarDrain = kBarSDP + 5;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kQMiscOff);
-  int* abort_flag = reinterpret_cast<int*>(smem + C::kQMiscOff + 4);
-  const WaitCtl ctl{abort_flag, p.timeout_ns};
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  // heaviest (last) query tiles first
-  const int per_tile = p.B * p.Hkv * p.NP;
-  const int qt = p.n_tiles - 1 - static_cast<int>(blockIdx.x) / per_tile;
-  int rem = static_cast<int>(blockIdx.x) % per_tile;
-  const int b = rem / (p.Hkv * p.NP);
-  rem %= p.Hkv * p.NP;
-  const int g = rem / p.NP;
-  const int h0 = g * p.G + (rem % p.NP) * p.Gp;
-  const int tpt = 128 / p.Gp;
-  const int tok0 = qt * tpt;
-  // key tiles: the band of the tile's first and last tokens
-  const int first = tok0, last = min(tok0 + tpt, p.Sq) - 1;
-  const int off = p.Skv - p.Sq;
-  int jlo = 0, jhi = 0;
-  {
-    const int lo = p.window > 0 ? max(0, first + off - p.window + 1) : 0;
-    const int hi = p.causal ? min(last + off, p.Skv - 1) : p.Skv - 1;
-    if (hi >= lo && hi >= 0) {
-      jlo = lo / 128;
-      jhi = hi / 128 + 1;
-    }
-  }
-  const int n_kt = jhi - jlo;
-
-  if (threadIdx.x == 0) {
-    for (int x = 0; x < C::kQNumBars; ++x)
-      mbar_init(bar(x), (x == kBarFree || x == kBarDS) ? 256 : 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 9) {
-    tmem_alloc(smem_u32(tmem_holder), C::kTmemCols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
-  constexpr uint32_t colS = 0, colDP = 128, colDQ = 256, colDS = 384;
-
-  if (warp == 8) {
-    // ============ producer ============
-    if (lane == 0 && n_kt > 0) {
-      // (with no key tile the epilogue writes zeros into the Q tile: nothing may land there)
-      mbar_arrive_expect_tx(bar(kBarIn), 2 * C::kTileBytes);
-#pragma unroll
-      for (int hf = 0; hf < C::kHalves; ++hf) {
-        tma_load_4d(sb + C::kQOff + hf * C::kAtomBytes, &tm_q, bar(kBarIn), 64 * hf, h0, tok0, b);
-        tma_load_4d(sb + C::kDOOff + hf * C::kAtomBytes, &tm_do, bar(kBarIn), 64 * hf, h0, tok0, b);
-      }
-      int issued = 0;
-      bool ok = true;
-      for (int t = 0; t < n_kt && ok; ++t) {
-#pragma unroll
-        for (int kind = 0; kind < 2; ++kind) {
-          const int pos = 2 * t + kind;
-          const int s = pos % C::kQStages;
-          if (!mbar_wait(bar(kBarKVEmpty + s), ((pos / C::kQStages) & 1) ^ 1, ctl)) {
-            ok = false;
-            break;
-          }
-          // K(t) and V(t) land on the full barrier of K(t)'s stage (an even stage)
-          const int sf = (2 * t) % C::kQStages;
-          if (kind == 0) mbar_arrive_expect_tx(bar(kBarKVFull + sf), 2 * C::kTileBytes);
-#pragma unroll
-          for (int hf = 0; hf < C::kHalves; ++hf)
-            tma_load_4d(sb + C::kQKVOff + s * C::kTileBytes + hf * C::kAtomBytes,
-                        kind ? &tm_v : &tm_k, bar(kBarKVFull + sf), 64 * hf, g, 128 * (jlo + t), b);
-          issued = pos + 1;
-        }
-      }
-      volatile int zero = 0;
-      const WaitCtl drain_ctl{&zero, p.timeout_ns};
-      mbar_wait(bar(kBarIn), 0, drain_ctl);
-      for (int s = 0; s < C::kQStages && s < issued; s += 2) {
-        const int lastp = s + C::kQStages * ((issued - 1 - s) / C::kQStages);
-        mbar_wait(bar(kBarKVFull + s), (lastp / C::kQStages) & 1, drain_ctl);
-      }
-    }
-  } else if (warp == 9) {
-    // ============ MMA issuer ============
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false);
-      constexpr uint32_t idesc_acc = idesc_bf16_f32(128, D, true);
-      auto mma_rows = [&](uint32_t d, uint32_t a, uint32_t bt) {
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t o2 = (kk / 4) * C::kAtomBytes + (kk % 4) * 32;
-          umma_ss(tmem + d, smem_desc_sw128(a + o2, 16, 1024), smem_desc_sw128(bt + o2, 16, 1024),
-                  idesc_s, kk > 0 ? 1u : 0u);
-        }
-      };
-      // K(t) and V(t) in shared memory (one barrier for both).  The MMAs read them through
-      // the async proxy that wrote them; no tcgen05 fence is needed after this wait.
-      auto kv_wait = [&](int pos) {
-        return mbar_wait(bar(kBarKVFull + pos % C::kQStages), (pos / C::kQStages) & 1, ctl);
-      };
-      // Order: S(0) dP(0) | S(t+1) dP(t+1) once S(t), dP(t) are in registers | dQ(t) once
-      // dS(t) is in TMEM: the next tile's products overlap the elementwise work on this one.
-      auto tile_addr = [&](int pos) {
-        return sb + C::kQKVOff + (pos % C::kQStages) * C::kTileBytes;
-      };
-      auto issue_sdp = [&](int t) -> bool {
-        if (!kv_wait(2 * t)) return false;
-        mma_rows(colS, sb + C::kQOff, tile_addr(2 * t));       // S = Q K^T
-        mma_rows(colDP, sb + C::kDOOff, tile_addr(2 * t + 1));  // dP = dO V^T
-        tc_commit(bar(kBarSDP));
-        tc_commit(bar(kBarKVEmpty + (2 * t + 1) % C::kQStages));  // V(t) is done
-        return true;
-      };
-      bool ok = n_kt > 0 && mbar_wait(bar(kBarIn), 0, ctl);
-      tc_fence_after();
-      if (ok) ok = issue_sdp(0);
-      for (int t = 0; t < n_kt && ok; ++t) {
-        if (t + 1 < n_kt) {
-          if (!(ok = mbar_wait(bar(kBarFree), t & 1, ctl))) break;
-          tc_fence_after();
-          if (!(ok = issue_sdp(t + 1))) break;
-        }
-        if (!(ok = mbar_wait(bar(kBarDS), t & 1, ctl))) break;
-        tc_fence_after();
-        // dQ += dS K (K tile as the MN-major B operand)
-        const uint32_t kt = tile_addr(2 * t);
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tmem + colDQ, tmem + colDS + kk * 8,
-                  smem_desc_sw128(kt + kk * 16 * 128, C::kAtomBytes, 1024), idesc_acc,
-                  (t == 0 && kk == 0) ? 0u : 1u);
-        tc_commit(bar(kBarDQ));
-        tc_commit(bar(kBarKVEmpty + (2 * t) % C::kQStages));
-      }
-      tc_commit(bar(kBarO));
-      tc_commit(bar(kBarDrain));
-      volatile int zero = 0;
-      const WaitCtl drain_ctl{&zero, p.timeout_ns};
-      mbar_wait(bar(kBarDrain), 0, drain_ctl);
-    }
-  } else {
-    // ============ elementwise: thread = Q row; this warp's half of the key columns ============
-    const int wq = warp & 3, ch = warp >> 2;
-    const int r = 32 * wq + lane;
-    const int i = tok0 + r / p.Gp;
-    const int hh = h0 + r % p.Gp;
-    const uint32_t trow = tmem + (static_cast<uint32_t>(32 * wq) << 16);
-    const uint64_t sl2 = f2(p.scale_log2, p.scale_log2);
-    const size_t vrow = (static_cast<size_t>(b) * p.Hq + hh) * p.Sq_pad + min(i, p.Sq_pad - 1);
-    const float nl2 = p.lse2[vrow], ndl = p.delta[vrow];  // -L log2(e), -D
-    const uint64_t nl2x2 = f2(nl2, nl2), ndlx2 = f2(ndl, ndl);
-    const int ip = i + off;
-    const int my_lo = p.window > 0 ? max(0, ip - p.window + 1) : 0;
-    const int my_hi = p.causal ? min(ip, p.Skv - 1) : p.Skv - 1;
-    // rows of the tile that bound its masks (all rows of a tile share the key-tile range)
-    const int lo_last = p.window > 0 ? max(0, last + off - p.window + 1) : 0;
-    const int hi_first = p.causal ? min(first + off, p.Skv - 1) : p.Skv - 1;
-    for (int t = 0; t < n_kt; ++t) {
-      const int j = jlo + t;
-      bool ok = mbar_wait(bar(kBarSDP), t & 1, ctl);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      const bool need_mask = (128 * j < lo_last) || (128 * j + 127 > hi_first) || i >= p.Sq;
-      uint32_t ds[32];
-#pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
-        uint32_t sv[32], dv[32];
-        tmem_ld32(trow + colS + 64 * ch + 32 * cc, sv);
-        tmem_ld32(trow + colDP + 64 * ch + 32 * cc, dv);
-        tmem_wait_ld();
-#pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          float a0, a1;
-          f2_split(f2_fma(f2(__uint_as_float(sv[2 * x]), __uint_as_float(sv[2 * x + 1])), sl2,
-                          nl2x2), a0, a1);
-          float p0 = ex2(a0), p1 = ex2(a1);
-          if (need_mask) {
-            const int key = 128 * j + 64 * ch + 32 * cc + 2 * x;
-            if (key < my_lo || key > my_hi || i >= p.Sq) p0 = 0.f;
-            if (key + 1 < my_lo || key + 1 > my_hi || i >= p.Sq) p1 = 0.f;
-          }
-          float d0, d1;
-          f2_split(f2_mul(f2(p0, p1), f2_add(f2(__uint_as_float(dv[2 * x]),
-                                                 __uint_as_float(dv[2 * x + 1])), ndlx2)),
-                   d0, d1);
-          ds[16 * cc + x] = pack_bf16x2(d0, d1);
-        }
-      }
-      // S and dP of this tile have been read: the next tile's products may start
-      tc_fence_before();
-      mbar_arrive(bar(kBarFree));
-      // the previous dQ product has read its dS before this one is written over it
-      if (t > 0) {
-        ok = mbar_wait(bar(kBarDQ), (t - 1) & 1, ctl);
-        if (!__all_sync(0xffffffffu, ok)) break;
-        tc_fence_after();
-      }
-      tmem_st32(trow + colDS + 32 * ch, ds);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(kBarDS));
-    }
-    // ---- epilogue: scale * dQ -> bf16 -> swizzled smem (the Q tile) -> TMA; warps 0-3 take
-    // the first half of the head dims, warps 4-7 the second ----
-    bool have = false;
-    if (n_kt > 0) {
-      bool ok = mbar_wait(bar(kBarO), 0, ctl);
-      have = __all_sync(0xffffffffu, ok);
-      tc_fence_after();
-    }
-    uint8_t* stage = smem + C::kQOff;
-#pragma unroll
-    for (int cc = 0; cc < D / 64; ++cc) {
-      const int c = ch * (D / 64) + cc;
-      uint32_t ov[32];
-      if (have) {
-        tmem_ld32(trow + colDQ + 32 * c, ov);
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int x = 0; x < 32; ++x) ov[x] = 0u;
-      }
-      const int hf = c >> 1;
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint4 w;
-        w.x = pack_bf16x2(__uint_as_float(ov[8 * q4 + 0]) * p.scale, __uint_as_float(ov[8 * q4 + 1]) * p.scale);
-        w.y = pack_bf16x2(__uint_as_float(ov[8 * q4 + 2]) * p.scale, __uint_as_float(ov[8 * q4 + 3]) * p.scale);
-        w.z = pack_bf16x2(__uint_as_float(ov[8 * q4 + 4]) * p.scale, __uint_as_float(ov[8 * q4 + 5]) * p.scale);
-        w.w = pack_bf16x2(__uint_as_float(ov[8 * q4 + 6]) * p.scale, __uint_as_float(ov[8 * q4 + 7]) * p.scale);
-        const int chunk = ((c & 1) * 4 + q4) ^ (r & 7);
-        *reinterpret_cast<uint4*>(stage + hf * C::kAtomBytes + r * 128 + chunk * 16) = w;
-      }
-    }
-    fence_proxy_async_smem();
-    named_bar_sync(1, 256);
-    if (threadIdx.x == 0 && tok0 < p.Sq) {
-#pragma unroll
-      for (int hf = 0; hf < C::kHalves; ++hf)
-        tma_store_4d(&tm_dq, sb + C::kQOff + hf * C::kAtomBytes, 64 * hf, h0, tok0, b);
-      tma_store_commit();
-      tma_store_wait_read_all();
-    }
-  }
-
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 9) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem, C::kTmemCols);
-  }
+__global__ void __launch_bounds__(256) fa_bwd_dq_finalize_kernel(const float* acc, uint16_t* dq,
+                                                                 float scale, long long n8) {
+  const long long t = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
+  if (t >= n8) return;
+  const float4* a = reinterpret_cast<const float4*>(acc) + 2 * t;
+  const float4 x = a[0], y = a[1];
+  uint4 w;
+  w.x = pack_bf16x2(x.x * scale, x.y * scale);
+  w.y = pack_bf16x2(x.z * scale, x.w * scale);
+  w.z = pack_bf16x2(y.x * scale, y.y * scale);
+  w.w = pack_bf16x2(y.z * scale, y.w * scale);
+  reinterpret_cast<uint4*>(dq)[t] = w;
 }
 
 }  // namespace fa

@@ -176,13 +176,32 @@ int encode_f32_3d(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1, 
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
-int bwd_sq_pad(int Sq) { return (Sq + 127) / 128 * 128; }
-
-size_t bwd_ws_bytes(int B, int Hq, int Sq) {
-  return 2ull * static_cast<size_t>(B) * Hq * bwd_sq_pad(Sq) * sizeof(float);
+// fp32 [n3][n2][n1][n0] (n0 innermost), boxes of (32, 1, 32, 1) = 32 rows of 128 bytes,
+// 128-byte swizzle: the backward pass adds dQ tiles into its accumulator through it.
+int encode_f32_4d_rows32(CUtensorMap* map, const void* base, uint64_t n0, uint64_t n1,
+                         uint64_t n2, uint64_t n3) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return FA_ERR_CUDA;
+  const cuuint64_t dims[4] = {n0, n1, n2, n3};
+  const cuuint64_t strides[3] = {n0 * 4, n0 * n1 * 4, n0 * n1 * n2 * 4};
+  const cuuint32_t box[4] = {32, 1, 32, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
-std::atomic<uint64_t> g_attr_bwd[4];
+int bwd_sq_pad(int Sq) { return (Sq + 127) / 128 * 128; }
+
+// -L log2(e) and -D per padded row, then the fp32 dQ accumulator [B, Sq, Hq, 128] (sized for
+// the larger head dimension, so the size does not depend on D)
+size_t bwd_ws_bytes(int B, int Hq, int Sq) {
+  return 2ull * static_cast<size_t>(B) * Hq * bwd_sq_pad(Sq) * sizeof(float) +
+         static_cast<size_t>(B) * Sq * Hq * 128 * sizeof(float);
+}
+
+std::atomic<uint64_t> g_attr_bwd[2];
 
 template <int D>
 int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -209,9 +228,11 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   p.lse = lse;
   p.lse2 = static_cast<float*>(ws);
   p.delta = p.lse2 + static_cast<size_t>(B) * Hq * p.Sq_pad;
+  p.dq_acc = p.delta + static_cast<size_t>(B) * Hq * p.Sq_pad;
+  p.dq = static_cast<uint16_t*>(dq);
   p.timeout_ns = kKernelTimeoutNs;
 
-  // 1. D and L * log2(e)
+  // 1. D and L * log2(e); the dQ accumulator zeroed
   const long long rows = static_cast<long long>(B) * Hq * p.Sq_pad;
   const long long rows_per_block = 8 * (256 / D);  // 8 warps of 256 / D rows each
   const long long prep_blocks = (rows + rows_per_block - 1) / rows_per_block;
@@ -220,7 +241,7 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
 
   int rc;
-  CUtensorMap tk, tv, tq1, tdo1, tvec, tdk, tdv;
+  CUtensorMap tk, tv, tq1, tdo1, tvec, tdk, tdv, tdqa;
   if ((rc = encode_bf16_4d(&tk, k, D, Hkv, Skv, B, 1, 128)) != FA_OK) return rc;
   if ((rc = encode_bf16_4d(&tv, v, D, Hkv, Skv, B, 1, 128)) != FA_OK) return rc;
   if ((rc = encode_bf16_4d(&tq1, q, D, Hq, Sq, B, 1, 128)) != FA_OK) return rc;
@@ -229,32 +250,25 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
     return rc;
   if ((rc = encode_bf16_4d(&tdk, dk, D, Hkv, Skv, B, 1, 128)) != FA_OK) return rc;
   if ((rc = encode_bf16_4d(&tdv, dv, D, Hkv, Skv, B, 1, 128)) != FA_OK) return rc;
+  if ((rc = encode_f32_4d_rows32(&tdqa, p.dq_acc, D, Hq, Sq, B)) != FA_OK) return rc;
 
-  // 2. dK, dV: one CTA per (b, KV head, key tile)
+  // 2. dK, dV and the dQ shares: one CTA per (b, KV head, key tile)
   p.n_tiles = (Skv + 127) / 128;
   const long long grid_kv = static_cast<long long>(p.n_tiles) * B * Hkv;
   if (grid_kv > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
-  auto kdkdv = fa::fa_bwd_dkdv_kernel<D>;
-  if ((rc = ensure_smem_attr(kdkdv, C::kUSmemBytes, g_attr_bwd[D == 128 ? 0 : 1])) != FA_OK)
+  auto kbwd = fa::fa_bwd_kernel<D>;
+  if ((rc = ensure_smem_attr(kbwd, C::kUSmemBytes, g_attr_bwd[D == 128 ? 0 : 1])) != FA_OK)
     return rc;
-  kdkdv<<<static_cast<unsigned>(grid_kv), C::kThreads, C::kUSmemBytes, stream>>>(
-      tq1, tk, tv, tdo1, tvec, tdk, tdv, p);
+  kbwd<<<static_cast<unsigned>(grid_kv), C::kThreads, C::kUSmemBytes, stream>>>(
+      tq1, tk, tv, tdo1, tvec, tdk, tdv, tdqa, p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
 
-  // 3. dQ: one CTA per 128-row Q tile (query heads packed into rows as in the forward pass)
-  const uint32_t tpt = 128 / p.Gp;
-  CUtensorMap tq, tdo, tdq;
-  if ((rc = encode_bf16_4d(&tq, q, D, Hq, Sq, B, p.Gp, tpt)) != FA_OK) return rc;
-  if ((rc = encode_bf16_4d(&tdo, dout, D, Hq, Sq, B, p.Gp, tpt)) != FA_OK) return rc;
-  if ((rc = encode_bf16_4d(&tdq, dq, D, Hq, Sq, B, p.Gp, tpt)) != FA_OK) return rc;
-  p.n_tiles = (Sq + static_cast<int>(tpt) - 1) / static_cast<int>(tpt);
-  const long long grid_q = static_cast<long long>(p.n_tiles) * B * Hkv * p.NP;
-  if (grid_q > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
-  auto kdq = fa::fa_bwd_dq_kernel<D>;
-  if ((rc = ensure_smem_attr(kdq, C::kQSmemBytes, g_attr_bwd[D == 128 ? 2 : 3])) != FA_OK)
-    return rc;
-  kdq<<<static_cast<unsigned>(grid_q), C::kThreads, C::kQSmemBytes, stream>>>(tq, tk, tv, tdo,
-                                                                              tdq, p);
+  // 3. dQ = scale * accumulator, bf16
+  const long long n8 = static_cast<long long>(B) * Sq * Hq * D / 8;
+  const long long fin_blocks = (n8 + 255) / 256;
+  if (fin_blocks > 0x7fffffffLL) return FA_ERR_INVALID_ARG;
+  fa::fa_bwd_dq_finalize_kernel<<<static_cast<unsigned>(fin_blocks), 256, 0, stream>>>(
+      p.dq_acc, p.dq, scale, n8);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -11,11 +11,12 @@
 
 namespace fa {
 
-// Device-side status word.  Kernels OR these bits in when a bounded wait gives up, or when an
-// index read from device memory (a page id, a sequence length) is out of range; the host reads
-// and clears it in fa_device_status().  The library is built as a single translation unit, so
-// the definition lives here.
-enum : unsigned { kDevStatusTimeout = 1u, kDevStatusBadIndex = 2u };
+// Device-side status word.  Kernels OR these bits in when a bounded wait gives up, when an
+// index read from device memory (a page id, a sequence length) is out of range, or when the
+// shared memory they were given is not aligned as they need; the host reads and clears it in
+// fa_device_status().  The library is built as a single translation unit, so the definition
+// lives here.
+enum : unsigned { kDevStatusTimeout = 1u, kDevStatusBadIndex = 2u, kDevStatusLayout = 4u };
 __device__ unsigned int g_fa_device_status = 0;
 // Where status_take_kernel leaves the word it took, for the host to read after a sync.
 __device__ unsigned int g_fa_status_taken = 0;
@@ -120,6 +121,17 @@ __device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t sr
                                              int c2, int c3) {
   asm volatile(
       "cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::
+          "l"(reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+
+// Element-wise add of a shared-memory box into a 4-D global tensor (the tensor map's type),
+// tracked by the bulk-group of the issuing thread like a store.
+__device__ __forceinline__ void tma_reduce_add_4d(const CUtensorMap* map, uint32_t src, int c0,
+                                                  int c1, int c2, int c3) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::
           "l"(reinterpret_cast<uint64_t>(map)),
       "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
