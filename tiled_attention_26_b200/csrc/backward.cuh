@@ -482,9 +482,12 @@ __global__ void __launch_bounds__(320, 1)
       tmem_wait_ld();
       tc_fence_before();
       mbar_arrive(bar(kBarDQFree));
-      // the staging below overwrites Q and dS^T, which dK += dS^T Q reads
-      ok = mbar_wait(bar(kBarDKDone), u & 1, ctl);
-      if (!__all_sync(0xffffffffu, ok)) break;
+      // the staging of ch = 1 goes over dS^T, which dK += dS^T Q reads (ch = 0 stages over dO,
+      // which dP and dV finished reading before dS was computed)
+      if (ch) {
+        ok = mbar_wait(bar(kBarDKDone), u & 1, ctl);
+        if (!__all_sync(0xffffffffu, ok)) break;
+      }
       {
         // Stage this warp's 32 rows x D/2 dims: boxes of 32 rows x 32 fp32 (128 bytes a row,
         // 128-byte swizzle), box (wq, k) at 4 KB * (k * 4 + wq) of the unit's dO tile (ch = 0)
