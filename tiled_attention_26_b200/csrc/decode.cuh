@@ -325,6 +325,9 @@ __global__ void __launch_bounds__(160, kBits == 8 ? 3 : 1) fa_decode_split_kerne
     // scales by bulk copies whenever their rows are 16-byte aligned: page scale rows always
     // are (page_size >= 16); contiguous rows when Skv is a multiple of 4
     const bool bulk_scales = kPaged || (p.Skv % 4 == 0);
+    // the K/V codes are read once per call: evict them first, so that streaming the cache does
+    // not push the rest of a serving step's working set (a prefill's K/V, say) out of L2
+    const uint64_t stream_pol = l2_evict_first_policy();
     int issued = 0;
     for (int i = 0; i < n_stages; ++i) {
       const int s = i % C::kStages;
@@ -347,14 +350,14 @@ __global__ void __launch_bounds__(160, kBits == 8 ? 3 : 1) fa_decode_split_kerne
               // a box past the split's last key reads the split's last page
               const int pg = page_of(min(t, t_end - 1));
               const int r0 = t & pmask;
-              tma_load_4d(kt + off, &tm_k, bar_full(s), 0, kvh, r0, pg);
-              tma_load_4d(vt + off, &tm_v, bar_full(s), 0, kvh, r0, pg);
+              tma_load_4d_policy(kt + off, &tm_k, bar_full(s), 0, kvh, r0, pg, stream_pol);
+              tma_load_4d_policy(vt + off, &tm_v, bar_full(s), 0, kvh, r0, pg, stream_pol);
               const size_t idx = ((static_cast<size_t>(pg) * p.Hkv + kvh) << p.page_shift) + r0;
               bulk_g2s(ks_dst + 4 * (t - t0), p.k_scale + idx, 4 * box_t, bar_full(s));
               bulk_g2s(vs_dst + 4 * (t - t0), p.v_scale + idx, 4 * box_t, bar_full(s));
             } else {
-              tma_load_4d(kt + off, &tm_k, bar_full(s), 0, kvh, t, b);
-              tma_load_4d(vt + off, &tm_v, bar_full(s), 0, kvh, t, b);
+              tma_load_4d_policy(kt + off, &tm_k, bar_full(s), 0, kvh, t, b, stream_pol);
+              tma_load_4d_policy(vt + off, &tm_v, bar_full(s), 0, kvh, t, b, stream_pol);
             }
           }
           if constexpr (!kPaged) {
@@ -373,8 +376,8 @@ __global__ void __launch_bounds__(160, kBits == 8 ? 3 : 1) fa_decode_split_kerne
           const uint32_t kt = sb + s * C::kStageBytes, vt = kt + C::kTile;
           for (int t = t0; t < t0 + C::kT; t += box_t) {
             const uint32_t off = (t - t0) * C::kRow;
-            tma_load_4d(kt + off, &tm_k, bar_full(s), 0, kvh, t, b);
-            tma_load_4d(vt + off, &tm_v, bar_full(s), 0, kvh, t, b);
+            tma_load_4d_policy(kt + off, &tm_k, bar_full(s), 0, kvh, t, b, stream_pol);
+            tma_load_4d_policy(vt + off, &tm_v, bar_full(s), 0, kvh, t, b, stream_pol);
           }
         }
 #pragma unroll
