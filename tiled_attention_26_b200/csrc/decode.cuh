@@ -47,6 +47,10 @@
 
 namespace fa {
 
+// The paged kernel orders its CTAs by sequence length when the batch has at most this many
+// sequences (one per thread of a CTA).
+constexpr int kDecodeRankMaxB = 128;
+
 struct DecodeParams {
   const uint16_t* q;  // bf16 [B, 1, Hq, D]
   const int8_t* k;    // [B, Skv, Hkv, D]; paged: [num_pages, P, Hkv, D]
@@ -261,7 +265,33 @@ __global__ void __launch_bounds__(160, kBits == 8 ? 3 : 1) fa_decode_split_kerne
   // same time stream the same key rows (all KV heads of a key are contiguous in memory).
   const int kvh = blockIdx.x, split = blockIdx.y;
   const int nhb = (p.G + 7) / 8;
-  const int b = static_cast<int>(blockIdx.z) / nhb, hb = static_cast<int>(blockIdx.z) % nhb;
+  int b = static_cast<int>(blockIdx.z) / nhb;
+  const int hb = static_cast<int>(blockIdx.z) % nhb;
+  if constexpr (kPaged) {
+    // Longest sequences first: with mixed lengths a split's work is proportional to its
+    // sequence's length, and CTAs start in grid order, so the long ones go in the first wave
+    // rather than the last.  CTA rank r takes the sequence of length rank r (ties by index);
+    // each thread ranks one sequence (up to kDecodeRankMaxB sequences; larger batches keep their
+    // order).  Lengths are clamped as below, so a bad one cannot break the permutation.
+    __shared__ int s_len[kDecodeRankMaxB];
+    __shared__ int s_b;
+    if (p.B <= kDecodeRankMaxB) {
+      const int cap = p.max_pages << p.page_shift;
+      if (threadIdx.x < p.B) s_len[threadIdx.x] = max(0, min(p.seqlens[threadIdx.x], cap));
+      __syncthreads();
+      if (threadIdx.x < p.B) {
+        const int me = threadIdx.x, lme = s_len[me];
+        int rank = 0;
+        for (int x = 0; x < p.B; ++x) {
+          const int lx = s_len[x];
+          rank += (lx > lme || (lx == lme && x < me)) ? 1 : 0;
+        }
+        if (rank == b) s_b = me;
+      }
+      __syncthreads();
+      b = s_b;
+    }
+  }
   const int head0 = kvh * p.G + hb * 8;
   const int nheads = min(8, p.G - hb * 8);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
