@@ -50,6 +50,11 @@ PAGED = [
     (2, 4, 4, 64, 256, [777, 256], 5),             # MHA, large pages
     (4, 8, 2, 128, 64, [0, 5, 0, 70], 4),          # empty sequences: O = 0, LSE = -inf
     (1, 8, 2, 128, 16, [5], 16),                   # more splits than groups
+    # lengths ranked on the device: equal lengths (ties by index), ascending order
+    (6, 8, 2, 128, 16, [48, 200, 48, 7, 200, 48], 3),
+    (5, 4, 1, 64, 16, [10, 20, 30, 40, 50], 2),
+    # more sequences than the kernel ranks (one per thread): grid order is kept
+    (130, 4, 1, 64, 16, [(7 * x) % 50 for x in range(130)], 2),
 ]
 
 
