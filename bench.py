@@ -48,13 +48,13 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # dram__bytes_read.sum + dram__bytes_write.sum per launch from ncu, keyed by the sha256 of the
 # kernel sources they were taken on; a kernel edited since then reports traffic = null.
 NCU_TRAFFIC = {
-    # profiles/fa_prefill_kernel_mha_causal.md: 534,377,472 B read + 48,006,144 B written
-    "prefill": {"753bf7e28f87f0e5": 582_383_616},
-    # profiles/fa_decode_split_kernel_decode_int8.md: 1,108,583,680 B read + 14,467,328 B written
-    "decode": {"db2267d0a6c42aac": 1_123_051_008},
-    # profiles/fa_decode_split_kernel_decode_int8_paged.md: 424,287,744 B read + 4,637,696 B
+    # profiles/fa_prefill_kernel_mha_causal.md: 536,197,888 B read + 48,389,376 B written
+    "prefill": {"9a69e24198021cef": 584_587_264},
+    # profiles/fa_decode_split_kernel_decode_int8.md: 1,108,619,776 B read + 4,625,664 B written
+    "decode": {"fdcac03dd1d0d86e": 1_113_245_440},
+    # profiles/fa_decode_split_kernel_decode_int8_paged.md: 424,227,840 B read + 3,291,904 B
     # written
-    "paged_decode": {"db2267d0a6c42aac": 428_925_440},
+    "paged_decode": {"fdcac03dd1d0d86e": 427_519_744},
 }
 
 
