@@ -59,6 +59,9 @@ CASES = [
     (1, 4, 4, 384, 384, 64, 1, 96),       # window, D=64
     (2, 16, 2, 160, 160, 128, 0, 0),      # G=8 packed rows, non-causal
     (1, 2, 1, 100, 40, 128, 1, 0),        # Sq > Skv: rows without keys
+    (1, 16, 1, 130, 257, 64, 1, 0),       # G = 16, D = 64, Sq != Skv, ragged key tail
+    (2, 4, 2, 129, 129, 128, 1, 64),      # window, one row past a tile, two batches
+    (1, 2, 2, 1000, 1000, 128, 0, 0),     # non-causal, eight key tiles per query tile
 ]
 
 
